@@ -1,0 +1,157 @@
+/*
+ * mlra.h - C ABI of the B200 (sm_100a) decode path for Multi-Head Low-Rank Attention.
+ *
+ * The operation (one decode step, one new query token per sequence):
+ *   Each cached token holds one latent c = [c_1 | ... | c_k] cut into k blocks of width
+ *   d_b = d_c / k, plus one decoupled RoPE key k^R of width d_rope shared by every head
+ *   ("Multi-Head Low-Rank Attention: Making Compressed Attention Actually Parallelizable",
+ *   Core Mechanism and Framework Shift; "Multi-Head Low-Rank Attention" abstract). Head group
+ *   j = heads [j*h/k, (j+1)*h/k) attends only to block c_j. For head h in group j:
+ *     q~_h  = (W^UK_h)^T q^C_h                       query absorption (lesty.tech MLA article,
+ *                                                    section 5; ai360xpert "Absorbing the
+ *                                                    up-projection")
+ *     s_t   = scale * (q~_h . c_j[t] + q^R_h . k^R[t])   decoupled RoPE score (lesty.tech, section 4)
+ *     o~_h  = sum_t softmax(s)_t c_j[t]               value accumulated in latent space
+ *     o_h   = W^UV_h o~_h                             one final up-projection (lesty.tech, section 5)
+ *   k = 1 is plain MLA (lesty.tech sections 3-5; Table 1 of the MLRA paper page, MLA row).
+ *
+ * Conventions shared by every entry point:
+ *   - Device pointers are CUDA global memory on the current device; host pointers are marked.
+ *   - The caller owns every buffer. The library allocates no device memory: scratch lives in
+ *     the caller's workspace (mlra_workspace_size). A handle borrows the weight pointers
+ *     until mlra_destroy.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream). No entry
+ *     point synchronises, except mlra_get_status.
+ *   - Return values are mlra_status codes. Argument errors are found on the host before any
+ *     launch. Errors that only the device can see (a page id outside the pool, a sequence
+ *     longer than its page-table row, a pipeline wait that timed out) are written to a
+ *     device status word that mlra_get_status reads after the stream has been synchronised.
+ *     No kernel traps.
+ *   - Calls on different streams are safe when each uses its own workspace.
+ *   - All symbol names are plain ASCII.
+ */
+#ifndef MLRA_H_
+#define MLRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLRA_OK = 0,
+  MLRA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, inconsistent dims */
+  MLRA_ERR_UNSUPPORTED = -2,   /* dims outside the compiled kernel set, or not an sm_100 GPU */
+  MLRA_ERR_CUDA = -3,          /* a CUDA runtime call failed */
+  MLRA_ERR_PAGE_OOB = -4,      /* device: a page-table entry outside [0, num_pages) */
+  MLRA_ERR_TIMEOUT = -5,       /* device: a pipeline wait passed its time limit */
+  MLRA_ERR_WORKSPACE = -6,     /* workspace smaller than mlra_workspace_size */
+  MLRA_ERR_SEQ_LEN = -7        /* device: seq_len < 0 or > pt_stride * page_size */
+} mlra_status;
+
+typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype;
+
+/* Problem dimensions, in the pages' notation. */
+typedef struct {
+  int h;               /* query heads */
+  int d_h;             /* head dim (width of q^C_h, K_h, V_h, o_h) */
+  int d_c;             /* latent width over all k blocks */
+  int d_rope;          /* decoupled RoPE key width d_h^R */
+  int k;               /* latent blocks; 1 = MLA. k must divide d_c and h */
+  int page_size;       /* tokens per cache page; must be 64 */
+  float softmax_scale; /* <= 0 selects 1/sqrt(d_h + d_rope) (a reading: the pages fix none) */
+} mlra_config;
+
+/* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, h/k, d_h):
+ *   (32, 16, <=16, 32), (128, 64, <=32, 128), (256, 64, <=64, 128); batch <= 4096. */
+
+typedef struct mlra_ctx* mlra_handle;
+
+/* Creates a handle. w_uk, w_uv: device bf16 [h][d_c/k][d_h], row-major: W^UK_h maps a
+ * block latent to a key by K_h[d] = sum_c c[c] * w_uk[h][c][d] (the ai360xpert code's
+ * (H, d_c, d_head) convention restricted to the head's block); likewise w_uv for values.
+ * Borrowed, must stay valid and unchanged until mlra_destroy. *out receives the handle. */
+int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra_handle* out);
+
+/* Releases the handle (host memory only). NULL-safe. */
+void mlra_destroy(mlra_handle h);
+
+/* Bytes of device workspace mlra_decode needs for `batch` sequences (host output). */
+int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes);
+
+/* One decode step for `batch` sequences.
+ *   q          device [batch][h][d_h + d_rope], q^C_h then q^R_h (already rotated),
+ *              dtype q_dtype (F32 or BF16; converted to bf16 for the tensor cores).
+ *   pool       device bf16 [num_pages][page_size][d_c + d_rope]: token row = [c_1..c_k | k^R].
+ *              16-byte aligned. Slots past a sequence's length may hold anything.
+ *   page_table device int32 [batch][pt_stride]: token t of sequence b lives in slot
+ *              t % page_size of page page_table[b*pt_stride + t/page_size].
+ *   seq_lens   device int32 [batch], 0 <= n_b <= pt_stride * page_size. n_b = 0 gives
+ *              o = 0 and lse = -inf.
+ *   out        device [batch][h][d_h], dtype out_dtype.
+ *   lse        device fp32 [batch][h] natural-log log-sum-exp of the scaled scores, or NULL.
+ *   workspace  device, >= mlra_workspace_size(batch) bytes, 256-byte aligned. Its first
+ *              4 bytes become this call's status word.
+ * Launches three kernels on `stream`: query absorption, split-KV latent attention, and
+ * log-sum-exp combine fused with the W^UV up-projection. */
+int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                int num_pages, const int32_t* page_table, int pt_stride,
+                const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
+                float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* Same as mlra_decode but stops before the up-projection: latent_out receives the
+ * normalised latent output o~ as device fp32 [batch][h][d_c/k], lse as above (nullable).
+ * For testing the attention and indexing stages on their own. */
+int mlra_decode_latent(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                       int num_pages, const int32_t* page_table, int pt_stride,
+                       const int32_t* seq_lens, int batch, float* latent_out, float* lse,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Writes new cache rows: token i goes to sequence seq_ids[i] at position positions[i], i.e.
+ * slot positions[i] % page_size of page page_table[seq_ids[i]*pt_stride + positions[i]/page_size].
+ *   c_new   device [n_tokens][d_c], kr_new device [n_tokens][d_rope], dtype in_dtype;
+ *           F32 input is rounded to bf16 to nearest-even.
+ *   page_table has `batch` rows of pt_stride entries; seq_ids[i] must be < batch.
+ *   status  device int32 word that receives a device error code (first error wins), or NULL.
+ * Rows whose page id falls outside [0, num_pages), or whose sequence / position falls outside
+ * the page table, are skipped and reported (MLRA_ERR_PAGE_OOB / MLRA_ERR_SEQ_LEN). */
+int mlra_append_cache(mlra_handle h, void* pool, int num_pages, const int32_t* page_table,
+                      int pt_stride, int batch, const int32_t* seq_ids, const int32_t* positions,
+                      const void* c_new, const void* kr_new, mlra_dtype in_dtype,
+                      int n_tokens, int32_t* status, void* stream);
+
+/* Runs the device split planner on seq_lens and writes the segments it would process:
+ * segments device int32 [max_segments][5] rows (b, group, tile_begin, tile_end, slot),
+ * count device int32. A group is a set of CTAs that shares one run of 128-token tiles;
+ * the rule is documented in mlra_get_info's comment. For bit-exact tests of the plan. */
+int mlra_plan(mlra_handle h, const int32_t* seq_lens, int batch, int pt_stride,
+              int32_t* segments, int max_segments, int32_t* count, void* stream);
+
+typedef struct {
+  int num_sms;         /* SMs of the handle's device */
+  int groups;          /* CTA groups of the decode kernel (floor(num_sms / ctas_per_group)) */
+  int ctas_per_group;  /* one CTA per (latent block, head chunk) */
+  int heads_per_cta;   /* query heads one CTA serves (padded to the MMA width) */
+  int tile_tokens;     /* 128: split granularity. Plan rule: tiles_b = ceil(n_b/128),
+                          T = sum tiles_b, quota = ceil(T/groups), group g takes flattened
+                          tiles [g*quota, min((g+1)*quota, T)), partial slot = b + g. */
+  int stages;          /* shared-memory pipeline depth of the decode kernel */
+  float softmax_scale; /* the scale in use */
+} mlra_info;
+
+int mlra_get_info(mlra_handle h, mlra_info* out);
+
+/* Copies a device status word (the first 4 bytes of a decode workspace, or an append status
+ * word) to *out (host). Synchronous: call after the stream that wrote it has finished. */
+int mlra_get_status(const void* status_word, int* out);
+
+/* Static string for a status code. */
+const char* mlra_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLRA_H_ */

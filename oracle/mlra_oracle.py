@@ -60,10 +60,9 @@ def head_block(head: int, h: int, k: int) -> int:
 def gather_rows(pool: np.ndarray, page_table: np.ndarray, b: int, n: int) -> np.ndarray:
     """Cache rows [n][d_c + d_r] of sequence b: token t lives at page table entry t // 64,
     slot t % 64 (PagedAttention-style paging, as the MLRA index page's bibliography cites)."""
-    rows = np.empty((n, pool.shape[-1]), dtype=np.float64)
-    for t in range(n):
-        rows[t] = pool[int(page_table[b, t // PAGE_SIZE]), t % PAGE_SIZE]
-    return rows
+    t = np.arange(n)
+    pages = np.asarray(page_table[b])[t // PAGE_SIZE].astype(np.int64)
+    return np.asarray(pool[pages, t % PAGE_SIZE], dtype=np.float64)
 
 
 def _split(rows: np.ndarray, j: int, d_c: int, k: int):

@@ -1,0 +1,489 @@
+// mlra_api.cu - the C ABI declared in include/mlra.h: argument checks, workspace carving,
+// TMA tensor maps, and the launch sequence of one decode step
+//   absorb (q -> packed absorbed query)  ->  latent attention (split-KV, persistent)
+//   ->  combine + W^UV up-projection,
+// chained with programmatic dependent launch so each kernel's prologue (barrier set-up,
+// TMEM allocation, weight prefetch, split planning) overlaps the previous kernel's tail.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mlra.h"
+#include "aux_kernels.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "proj.cuh"
+
+using namespace mlra;
+
+namespace {
+
+// ---------------------------------------------------------------------------------------
+// Compiled kernel set. A variant fixes (d_b, d_rope, heads per CTA, d_h) and the decode
+// kernel's shared-memory pipeline.
+// ---------------------------------------------------------------------------------------
+enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kNumVariants };
+
+using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
+using DecMlra4 = DecodeShape<128, 64, 32, 4, 1, 2>;
+using DecMlra4q2 = DecodeShape<128, 64, 32, 3, 2, 2>;
+using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
+
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
+struct VariantDims {
+  int d_b, d_r, np, d_h;
+};
+constexpr VariantDims kDims[kNumVariants] = {{32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// 2-D bf16 tensor [rows][cols] (row stride in bytes), box [box_rows][box_cols].
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride,
+              uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_cols * 2),
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int nt_for(int batch) { return batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : 128; }
+
+}  // namespace
+
+struct mlra_ctx {
+  mlra_config cfg;
+  const void* w_uk;
+  const void* w_uv;
+  int device;
+  int num_sms;
+  Variant var;
+  int d_b, d_r, np, chunks, nsub, heads_block, groups, stages;
+  float scale;
+  CUtensorMap map_wuk;
+  CUtensorMap map_wuv;
+};
+
+namespace {
+
+// ----- per-variant launch helpers -----
+template <class Dec>
+cudaError_t prep_decode() {
+  return cudaFuncSetAttribute(mlra_decode_kernel<Dec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Dec::SMEM_BYTES);
+}
+template <int DB, int DH, int NT>
+cudaError_t prep_proj() {
+  using S = ProjShape<DB, DH, NT>;
+  cudaError_t e = cudaFuncSetAttribute(mlra_absorb_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       S::SMEM1);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(mlra_uproj_kernel<S, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           S::SMEM4);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(mlra_uproj_kernel<S, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              S::SMEM4);
+}
+template <int DB, int DH>
+cudaError_t prep_proj_all() {
+  cudaError_t e;
+  if ((e = prep_proj<DB, DH, 16>()) != cudaSuccess) return e;
+  if ((e = prep_proj<DB, DH, 32>()) != cudaSuccess) return e;
+  if ((e = prep_proj<DB, DH, 64>()) != cudaSuccess) return e;
+  return prep_proj<DB, DH, 128>();
+}
+
+// `attr` must outlive the launch call that uses the returned config.
+cudaLaunchConfig_t launch_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                              cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = grid;
+  c.blockDim = block;
+  c.dynamicSmemBytes = smem;
+  c.stream = s;
+  if (pdl) {
+    attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr->val.programmaticStreamSerializationAllowed = 1;
+    c.attrs = attr;
+    c.numAttrs = 1;
+  }
+  return c;
+}
+
+template <int DB, int DH, int NT>
+cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
+  using S = ProjShape<DB, DH, NT>;
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(128), S::SMEM1, s, false, &attr);
+  return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, pp);
+}
+template <int DB, int DH, int NT, bool LATENT>
+cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
+  using S = ProjShape<DB, DH, NT>;
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(128), S::SMEM4, s, true, &attr);
+  return cudaLaunchKernelEx(&c, mlra_uproj_kernel<S, LATENT>, h->map_wuv, pp);
+}
+template <int DB, int DH>
+cudaError_t dispatch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
+  switch (nt_for(batch)) {
+    case 16: return launch_absorb<DB, DH, 16>(h, pp, batch, s);
+    case 32: return launch_absorb<DB, DH, 32>(h, pp, batch, s);
+    case 64: return launch_absorb<DB, DH, 64>(h, pp, batch, s);
+    default: return launch_absorb<DB, DH, 128>(h, pp, batch, s);
+  }
+}
+template <int DB, int DH, bool LATENT>
+cudaError_t dispatch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
+  switch (nt_for(batch)) {
+    case 16: return launch_uproj<DB, DH, 16, LATENT>(h, pp, batch, s);
+    case 32: return launch_uproj<DB, DH, 32, LATENT>(h, pp, batch, s);
+    case 64: return launch_uproj<DB, DH, 64, LATENT>(h, pp, batch, s);
+    default: return launch_uproj<DB, DH, 128, LATENT>(h, pp, batch, s);
+  }
+}
+
+template <class Dec>
+cudaError_t launch_decode(const mlra_ctx* h, const CUtensorMap& mc, const CUtensorMap& mr,
+                          const CUtensorMap& mqc, const CUtensorMap& mqr, const DecodeParams& dp,
+                          cudaStream_t s) {
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->groups * h->nsub), dim3(192), Dec::SMEM_BYTES, s, true, &attr);
+  return cudaLaunchKernelEx(&c, mlra_decode_kernel<Dec>, mc, mr, mqc, mqr, dp);
+}
+
+struct Workspace {
+  int* status;
+  __nv_bfloat16* q_pack;
+  float* o_part;
+  float* lse_part;
+  size_t bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Workspace carve(const mlra_ctx* h, int batch, void* base) {
+  Workspace w;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  w.status = reinterpret_cast<int*>(p + off);
+  off += 256;
+  w.q_pack = reinterpret_cast<__nv_bfloat16*>(p + off);
+  off += align256((size_t)batch * h->nsub * h->np * (h->d_b + h->d_r) * 2);
+  const size_t slots = (size_t)batch + h->groups;
+  w.o_part = reinterpret_cast<float*>(p + off);
+  off += align256(slots * h->cfg.h * h->d_b * 4);
+  w.lse_part = reinterpret_cast<float*>(p + off);
+  off += align256(slots * h->cfg.h * 4);
+  w.bytes = off;
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
+               const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch, void* out,
+               mlra_dtype out_dtype, float* lse, float* latent_out, void* workspace, size_t ws_bytes,
+               void* stream, int inject_stall, unsigned long long wait_limit_ns) {
+  if (!h || !q || !pool || !page_table || !seq_lens || !workspace) return MLRA_ERR_INVALID_ARG;
+  if (!out && !latent_out) return MLRA_ERR_INVALID_ARG;
+  if (batch <= 0 || batch > 4096 || num_pages <= 0 || pt_stride <= 0) return MLRA_ERR_INVALID_ARG;
+  if ((q_dtype != MLRA_F32 && q_dtype != MLRA_BF16) || (out && out_dtype != MLRA_F32 && out_dtype != MLRA_BF16))
+    return MLRA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pool) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MLRA_ERR_INVALID_ARG;
+  if ((long long)num_pages * kPage > 0x7fffffffLL) return MLRA_ERR_UNSUPPORTED;
+  Workspace w = carve(h, batch, workspace);
+  if (ws_bytes < w.bytes) return MLRA_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MLRA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = h->cfg.d_c + h->d_r;
+
+  // tensor maps over this call's pool and packed-query buffers
+  const int cw = h->d_b < 64 ? h->d_b : 64, rw = h->d_r < 64 ? h->d_r : 64;
+  CUtensorMap mc, mr, mqc, mqr;
+  const uint64_t qrows = (uint64_t)batch * h->nsub * h->np;
+  if (!make_map(&mc, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, cw) ||
+      !make_map(&mr, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, rw) ||
+      !make_map(&mqc, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, h->np, cw) ||
+      !make_map(&mqr, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, h->np, rw))
+    return MLRA_ERR_CUDA;
+
+  ProjParams pp = {};
+  pp.q = q;
+  pp.q_f32 = q_dtype == MLRA_F32;
+  pp.q_pack = w.q_pack;
+  pp.qscale = h->scale * kLog2e;
+  pp.d_r = h->d_r;
+  pp.np = h->np;
+  pp.nsub = h->nsub;
+  pp.chunks = h->chunks;
+  pp.heads_block = h->heads_block;
+  pp.o_part = w.o_part;
+  pp.lse_part = w.lse_part;
+  pp.out = out;
+  pp.out_f32 = out_dtype == MLRA_F32;
+  pp.lse_out = lse;
+  pp.latent_out = latent_out;
+  pp.seq_lens = seq_lens;
+  pp.pt_stride = pt_stride;
+  pp.groups = h->groups;
+  pp.batch = batch;
+  pp.h = h->cfg.h;
+  pp.status = w.status;
+  pp.wait_limit_ns = wait_limit_ns;
+
+  DecodeParams dp = {};
+  dp.seq_lens = seq_lens;
+  dp.page_table = page_table;
+  dp.pt_stride = pt_stride;
+  dp.batch = batch;
+  dp.num_pages = num_pages;
+  dp.groups = h->groups;
+  dp.nsub = h->nsub;
+  dp.chunks = h->chunks;
+  dp.heads_block = h->heads_block;
+  dp.h = h->cfg.h;
+  dp.d_c = h->cfg.d_c;
+  dp.o_part = w.o_part;
+  dp.lse_part = w.lse_part;
+  dp.status = w.status;
+  dp.wait_limit_ns = wait_limit_ns;
+  dp.inject_stall = inject_stall;
+
+  cudaError_t e = cudaSuccess;
+  const bool latent = latent_out != nullptr;
+  switch (h->var) {
+    case kTiny:
+      e = dispatch_absorb<32, 32>(h, pp, batch, s);
+      if (e == cudaSuccess) e = launch_decode<DecTiny>(h, mc, mr, mqc, mqr, dp, s);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<32, 32, true>(h, pp, batch, s) : dispatch_uproj<32, 32, false>(h, pp, batch, s);
+      break;
+    case kMlra4:
+      e = dispatch_absorb<128, 128>(h, pp, batch, s);
+      if (e == cudaSuccess)
+        e = h->stages == 3 ? launch_decode<DecMlra4q2>(h, mc, mr, mqc, mqr, dp, s)
+                           : launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<128, 128, false>(h, pp, batch, s);
+      break;
+    case kMlra2:
+      e = dispatch_absorb<256, 128>(h, pp, batch, s);
+      if (e == cudaSuccess) e = launch_decode<DecMlra2>(h, mc, mr, mqc, mqr, dp, s);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<256, 128, false>(h, pp, batch, s);
+      break;
+    default:
+      return MLRA_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra_handle* out) {
+  if (!cfg || !w_uk || !w_uv || !out) return MLRA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const mlra_config& c = *cfg;
+  if (c.h <= 0 || c.d_h <= 0 || c.d_c <= 0 || c.d_rope <= 0 || c.k <= 0) return MLRA_ERR_INVALID_ARG;
+  if (c.d_c % c.k != 0 || c.h % c.k != 0) return MLRA_ERR_INVALID_ARG;
+  if (c.page_size != kPage) return MLRA_ERR_UNSUPPORTED;
+  if (!aligned16(w_uk) || !aligned16(w_uv)) return MLRA_ERR_INVALID_ARG;
+  const int d_b = c.d_c / c.k, hb = c.h / c.k;
+  int var = -1;
+  for (int v = 0; v < kNumVariants; ++v)
+    if (kDims[v].d_b == d_b && kDims[v].d_r == c.d_rope && kDims[v].d_h == c.d_h && hb <= kDims[v].np) var = v;
+  if (var < 0) return MLRA_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLRA_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MLRA_ERR_CUDA;
+  if (prop.major != 10) return MLRA_ERR_UNSUPPORTED;
+
+  mlra_ctx* h = new mlra_ctx();
+  h->cfg = c;
+  h->w_uk = w_uk;
+  h->w_uv = w_uv;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->var = static_cast<Variant>(var);
+  h->d_b = d_b;
+  h->d_r = c.d_rope;
+  h->np = kDims[var].np;
+  h->heads_block = hb;
+  h->chunks = (hb + h->np - 1) / h->np;
+  h->nsub = c.k * h->chunks;
+  h->groups = h->num_sms / h->nsub;
+  h->scale = c.softmax_scale > 0.f ? c.softmax_scale : 1.0f / std::sqrt((float)(c.d_h + c.d_rope));
+  h->stages = 0;
+
+  cudaError_t e = cudaSuccess;
+  switch (h->var) {
+    case kTiny:
+      e = prep_decode<DecTiny>();
+      if (e == cudaSuccess) e = prep_proj_all<32, 32>();
+      h->stages = DecTiny::STAGES;
+      break;
+    case kMlra4:
+      e = prep_decode<DecMlra4>();
+      if (e == cudaSuccess) e = prep_decode<DecMlra4q2>();
+      if (e == cudaSuccess) e = prep_proj_all<128, 128>();
+      h->stages = DecMlra4::STAGES;
+      break;
+    case kMlra2:
+      e = prep_decode<DecMlra2>();
+      if (e == cudaSuccess) e = prep_proj_all<256, 128>();
+      h->stages = DecMlra2::STAGES;
+      break;
+    default:
+      break;
+  }
+  if (e != cudaSuccess) {
+    delete h;
+    return MLRA_ERR_CUDA;
+  }
+  // weight tensor maps: [h * d_b rows][d_h cols]
+  const int aw = c.d_h < 64 ? c.d_h : 64;
+  const int nmt_rows = d_b >= 128 ? d_b : 128;
+  const uint32_t boxr1 = nmt_rows < 256 ? nmt_rows : 256;
+  const uint32_t boxr4 = d_b < 256 ? d_b : 256;
+  if (!make_map(&h->map_wuk, w_uk, (uint64_t)c.h * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr1, aw) ||
+      !make_map(&h->map_wuv, w_uv, (uint64_t)c.h * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr4, aw)) {
+    delete h;
+    return MLRA_ERR_CUDA;
+  }
+  *out = h;
+  return MLRA_OK;
+}
+
+void mlra_destroy(mlra_handle h) { delete h; }
+
+int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes) {
+  if (!h || !bytes || batch <= 0 || batch > 4096) return MLRA_ERR_INVALID_ARG;
+  *bytes = carve(h, batch, nullptr).bytes;
+  return MLRA_OK;
+}
+
+int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
+                const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch, void* out,
+                mlra_dtype out_dtype, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  if (!out) return MLRA_ERR_INVALID_ARG;
+  return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, out_dtype,
+                    lse, nullptr, workspace, ws_bytes, stream, 0, kWaitLimitNs);
+}
+
+int mlra_decode_latent(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
+                       const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch,
+                       float* latent_out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  if (!latent_out) return MLRA_ERR_INVALID_ARG;
+  return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, nullptr,
+                    MLRA_F32, lse, latent_out, workspace, ws_bytes, stream, 0, kWaitLimitNs);
+}
+
+int mlra_append_cache(mlra_handle h, void* pool, int num_pages, const int32_t* page_table, int pt_stride,
+                      int batch, const int32_t* seq_ids, const int32_t* positions, const void* c_new,
+                      const void* kr_new, mlra_dtype in_dtype, int n_tokens, int32_t* status, void* stream) {
+  if (!h || !pool || !page_table || !seq_ids || !positions || !c_new || !kr_new) return MLRA_ERR_INVALID_ARG;
+  if (n_tokens < 0 || num_pages <= 0 || pt_stride <= 0 || batch <= 0) return MLRA_ERR_INVALID_ARG;
+  if (in_dtype != MLRA_F32 && in_dtype != MLRA_BF16) return MLRA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLRA_OK;
+  const int warps = 8;
+  mlra_append_kernel<<<(n_tokens + warps - 1) / warps, warps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<__nv_bfloat16*>(pool), num_pages, page_table, pt_stride, batch, seq_ids, positions, c_new,
+      kr_new, in_dtype == MLRA_F32, n_tokens, h->cfg.d_c, h->d_r, status);
+  return cudaGetLastError() == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
+}
+
+int mlra_plan(mlra_handle h, const int32_t* seq_lens, int batch, int pt_stride, int32_t* segments,
+              int max_segments, int32_t* count, void* stream) {
+  if (!h || !seq_lens || !segments || !count || batch <= 0 || max_segments < 0 || pt_stride <= 0)
+    return MLRA_ERR_INVALID_ARG;
+  mlra_plan_kernel<<<1, 192, 0, static_cast<cudaStream_t>(stream)>>>(seq_lens, batch, pt_stride, h->groups,
+                                                                    segments, max_segments, count, nullptr);
+  return cudaGetLastError() == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
+}
+
+int mlra_get_info(mlra_handle h, mlra_info* out) {
+  if (!h || !out) return MLRA_ERR_INVALID_ARG;
+  out->num_sms = h->num_sms;
+  out->groups = h->groups;
+  out->ctas_per_group = h->nsub;
+  out->heads_per_cta = h->np;
+  out->tile_tokens = kTile;
+  out->stages = h->stages;
+  out->softmax_scale = h->scale;
+  return MLRA_OK;
+}
+
+int mlra_get_status(const void* status_word, int* out) {
+  if (!status_word || !out) return MLRA_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpy(&v, status_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLRA_ERR_CUDA;
+  *out = v;
+  return MLRA_OK;
+}
+
+const char* mlra_status_string(int code) {
+  switch (code) {
+    case MLRA_OK: return "ok";
+    case MLRA_ERR_INVALID_ARG: return "invalid argument";
+    case MLRA_ERR_UNSUPPORTED: return "unsupported dimensions or device";
+    case MLRA_ERR_CUDA: return "CUDA runtime error";
+    case MLRA_ERR_PAGE_OOB: return "page id outside the pool";
+    case MLRA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case MLRA_ERR_WORKSPACE: return "workspace too small";
+    case MLRA_ERR_SEQ_LEN: return "sequence length outside its page-table row";
+    default: return "unknown status";
+  }
+}
+
+// Test hook (not in the public header): a decode whose producer withholds its first tile, so
+// the consumer's bounded wait runs out after `wait_limit_ns` and the status word reports
+// MLRA_ERR_TIMEOUT. Used to check that a stalled pipeline ends with an error, not a hang.
+int mlra_test_decode_stalled(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                             int num_pages, const int32_t* page_table, int pt_stride,
+                             const int32_t* seq_lens, int batch, void* out, void* workspace,
+                             size_t ws_bytes, unsigned long long wait_limit_ns, void* stream) {
+  return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, MLRA_F32,
+                    nullptr, nullptr, workspace, ws_bytes, stream, 1, wait_limit_ns);
+}
+
+}  // extern "C"

@@ -1,0 +1,428 @@
+// proj.cuh - the two per-head projections around the latent attention kernel.
+//
+//   absorb:  q~_h = scale * log2(e) * (W^UK_h)^T q^C_h     (lesty.tech MLA article, section 5;
+//            ai360xpert "Absorbing the up-projection"), written as bf16 into the packed query
+//            [b][latent block][head][q~ | q^R] that the decode kernel streams; q^R is scaled
+//            the same way, so the decode kernel's scores come out in log2 units.
+//   uproj:   o_h = W^UV_h o~_h                              ("a single final matrix
+//            multiplication", lesty.tech section 5), where o~_h is first merged from the
+//            decode kernel's split partials by log-sum-exp.
+//
+// Both are one CTA per (head, batch tile): D^T[M x N] = A_h[M x K] * X_h[N x K]^T with the
+// per-head weight as the tcgen05 A operand (M = 128 rows of the weight's output dim; TMA
+// load) and the batch as N (16..128; filled by the CTA's threads, because the activation
+// side needs a dtype conversion or a merge on the way in). 128 threads: every warp reads one
+// TMEM lane quadrant in the epilogue.
+#pragma once
+
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace mlra {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct ProjParams {
+  // absorb
+  const void* q;      // [B][h][d_h + d_r]
+  int q_f32;          // 1: fp32 q, 0: bf16 q
+  __nv_bfloat16* q_pack;  // [B][nsub][NP][DB + DR]
+  float qscale;       // softmax scale * log2(e)
+  int d_r;
+  int np;             // heads per decode CTA (rows per q_pack block)
+  int nsub;           // decode CTAs per group
+  int chunks;         // head chunks per latent block
+  int heads_block;    // h / k
+  // uproj
+  const float* o_part;
+  const float* lse_part;
+  void* out;          // [B][h][d_h]
+  int out_f32;
+  float* lse_out;     // [B][h] natural log, nullable
+  float* latent_out;  // [B][h][DB] fp32 (combine-only mode)
+  const int* seq_lens;
+  int pt_stride;
+  int groups;
+  // common
+  int batch;
+  int h;
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+
+template <int DB_, int DH_, int NT_>
+struct ProjShape {
+  static constexpr int DB = DB_, DH = DH_, NT = NT_;
+  // absorb: A = W^UK_h [DB rows][DH cols], K-major, K split into swizzle-width regions
+  static constexpr int AW = DH < 64 ? DH : 64;
+  static constexpr int NKR = DH / AW;
+  static constexpr int AROWB = AW * 2;
+  static constexpr int NMT = DB >= 128 ? DB / 128 : 1;
+  static constexpr int A1_REG = round_up(NMT * 128 * AROWB, 1024);
+  static constexpr int B1_REG = round_up(NT * AROWB, 1024);
+  static constexpr int A1_BOXR = NMT * 128 < 256 ? NMT * 128 : 256;
+  static constexpr int A1_TX = NKR * NMT * 128 * AROWB;
+  static constexpr int SMEM1 = NKR * A1_REG + NKR * B1_REG + 1024 + 256;
+  static constexpr int TMEM1 = NMT * NT <= 32 ? 32 : NMT * NT <= 64 ? 64 : NMT * NT <= 128 ? 128 :
+                               NMT * NT <= 256 ? 256 : 512;
+  // uproj: A = (W^UV_h)^T, MN-major: atoms of AW output columns, each DB rows (K) deep
+  static constexpr int ATOM = round_up(DB * AROWB, 1024);
+  static constexpr int NATOM = DH / AW;  // real atoms; M = 128 repeats the last via LBO = 0
+  static constexpr uint32_t A4_LBO = DH >= 128 ? ATOM : 0;
+  static constexpr int A4_BOXR = DB < 256 ? DB : 256;
+  static constexpr int A4_TX = NATOM * DB * AROWB;
+  static constexpr int BW = DB < 64 ? DB : 64;  // õ regions (K-major)
+  static constexpr int NKB = DB / BW;
+  static constexpr int BROWB = BW * 2;
+  static constexpr int B4_REG = round_up(NT * BROWB, 1024);
+  static constexpr int SMEM4 = NATOM * ATOM + NKB * B4_REG + 1024 + 1024;
+  static constexpr int TMEM4 = NT <= 32 ? 32 : NT <= 64 ? 64 : 128;
+  static_assert(DH <= 128, "one M tile of head dim");
+};
+
+// ---------------------------------------------------------------------------------------
+// absorb
+// ---------------------------------------------------------------------------------------
+template <class Sh>
+__global__ void __launch_bounds__(128, 1)
+    mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const ProjParams p) {
+  constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* A = smem;
+  uint8_t* Bq = smem + Sh::NKR * Sh::A1_REG;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bq + Sh::NKR * Sh::B1_REG);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int head = blockIdx.x;
+  const int n0 = blockIdx.y * NT;
+  const int warp = warp_id(), lane = lane_id();
+  const int qw = DB + p.d_r;
+  const int hb = head % p.heads_block;
+  const int blk = head / p.heads_block;
+  const int sub = blk * p.chunks + hb / p.np;
+  const int prow = hb % p.np;
+
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.status) *p.status = 0;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, Sh::TMEM1);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_map(&map_wuk);
+    mbar_arrive_expect_tx(&bars[0], Sh::A1_TX);
+    const uint64_t pol = l2_policy_evict_first();
+    for (int kr = 0; kr < Sh::NKR; ++kr)
+      for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
+        tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW,
+                    head * DB + r0, pol);
+  }
+
+  // q^C_h for the batch tile -> bf16, K-major swizzled; q^R_h -> packed query (scaled)
+  for (int idx = threadIdx.x; idx < NT * (DH / 8); idx += 128) {
+    const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
+    const int b = n0 + bl;
+    float v[8];
+    if (b < p.batch) {
+      const size_t base = ((size_t)b * p.h + head) * (DH + p.d_r) + d8;
+      if (p.q_f32) {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + base);
+        const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+        v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+        v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+      } else {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + base));
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          v[2 * e] = f.x;
+          v[2 * e + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    }
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]);
+    w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]);
+    w.w = pack_bf16x2(v[6], v[7]);
+    const int kr = d8 / Sh::AW;
+    *reinterpret_cast<uint4*>(Bq + kr * Sh::B1_REG +
+                              swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
+  }
+  for (int idx = threadIdx.x; idx < NT * p.d_r; idx += 128) {
+    const int bl = idx / p.d_r, r = idx % p.d_r;
+    const int b = n0 + bl;
+    if (b >= p.batch) continue;
+    const size_t src = ((size_t)b * p.h + head) * (DH + p.d_r) + DH + r;
+    const float x = p.q_f32 ? __ldg(static_cast<const float*>(p.q) + src)
+                            : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p.q) + src));
+    p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow) * qw + DB + r] = __float2bfloat16_rn(x * p.qscale);
+  }
+  // rows of a head chunk that no head fills (h/k below the MMA width) are zero
+  if (hb == p.heads_block - 1 && prow == hb % p.np) {
+    const int pad = p.np - 1 - prow;
+    for (int idx = threadIdx.x; idx < NT * pad * qw; idx += 128) {
+      const int bl = idx / (pad * qw), rest = idx % (pad * qw);
+      const int b = n0 + bl;
+      if (b >= p.batch) continue;
+      p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow + 1 + rest / qw) * qw + rest % qw] =
+          __float2bfloat16_rn(0.f);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  if (warp == 0) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns));
+    if (ok) {
+      tc_fence_after();
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
+        constexpr int KPR = Sh::AW / 16;  // MMA K steps per region
+#pragma unroll
+        for (int mt = 0; mt < Sh::NMT; ++mt)
+#pragma unroll
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            const uint64_t a = smem_desc(smem_u32(A + (ks / KPR) * Sh::A1_REG + mt * 128 * Sh::AROWB +
+                                                  (ks % KPR) * 32),
+                                         16, 8 * Sh::AROWB, swizzle_code(Sh::AROWB));
+            const uint64_t b = smem_desc(smem_u32(Bq + (ks / KPR) * Sh::B1_REG + (ks % KPR) * 32), 16,
+                                         8 * Sh::AROWB, swizzle_code(Sh::AROWB));
+            umma_bf16(tbase + mt * NT, a, b, idesc, ks > 0 ? 1u : 0u);
+          }
+        umma_commit(&bars[1]);
+      }
+      __syncwarp();
+    }
+  }
+  const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+    for (int mt = 0; mt < Sh::NMT; ++mt) {
+      const int c = mt * 128 + warp * 32 + lane;
+      float v[NT];
+      tmem_load_row<NT>(tbase + lane_base + mt * NT, v);
+      tmem_ld_wait();
+      if (c < DB) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const int b = n0 + n;
+          if (b < p.batch)
+            p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow) * qw + c] =
+                __float2bfloat16_rn(v[n] * p.qscale);
+        }
+      }
+    }
+  }
+  // drain before releasing TMEM and shared memory
+  if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
+  grid_launch_dependents();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Sh::TMEM1);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// combine + uproj (LATENT_ONLY: combine and write o~ in fp32, no projection)
+// ---------------------------------------------------------------------------------------
+template <class Sh, bool LATENT_ONLY>
+__global__ void __launch_bounds__(128, 1)
+    mlra_uproj_kernel(const __grid_constant__ CUtensorMap map_wuv, const ProjParams p) {
+  constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* A = smem;
+  uint8_t* Bo = smem + Sh::NATOM * Sh::ATOM;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bo + Sh::NKB * Sh::B4_REG);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* err_flag = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
+  int* scratch = reinterpret_cast<int*>(tmem_slot + 4);  // 40 ints
+  int* pref = scratch + 40;                              // NT ints
+
+  const int head = blockIdx.x;
+  const int n0 = blockIdx.y * NT;
+  const int warp = warp_id(), lane = lane_id();
+  const int cap_len = p.pt_stride * kPage;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    *err_flag = 0;
+    fence_mbar_init();
+  }
+  if (!LATENT_ONLY && warp == 0) {
+    tmem_alloc(tmem_slot, Sh::TMEM4);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = LATENT_ONLY ? 0u : *tmem_slot;
+
+  // the weight does not depend on the previous kernel: load it before waiting for it
+  if (!LATENT_ONLY && threadIdx.x == 0) {
+    tma_prefetch_map(&map_wuv);
+    mbar_arrive_expect_tx(&bars[0], Sh::A4_TX);
+    const uint64_t pol = l2_policy_evict_first();
+    for (int a = 0; a < Sh::NATOM; ++a)
+      for (int r0 = 0; r0 < DB; r0 += Sh::A4_BOXR)
+        tma_load_2d(A + a * Sh::ATOM + r0 * Sh::AROWB, &map_wuv, &bars[0], a * Sh::AW,
+                    head * DB + r0, pol);
+  }
+
+  // plan: total tiles and the flattened start of each sequence of this batch tile
+  int err = 0;
+  const int T = block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
+  const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
+  {
+    int running = 0;
+    for (int base = 0; base < min(p.batch, n0 + NT); base += blockDim.x) {
+      const int b = base + threadIdx.x;
+      const int t = b < p.batch ? tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err)) : 0;
+      int chunk_total;
+      const int pb = running + block_scan_tiles(t, scratch, &chunk_total);
+      if (b >= n0 && b < n0 + NT) pref[b - n0] = pb;
+      running += chunk_total;
+    }
+  }
+  if (err) atomicOr(err_flag, 1);
+  __syncthreads();
+
+  grid_dependency_wait();  // the partials come from the decode kernel
+
+  // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major)
+  constexpr int PER = DB / 32;  // features per lane
+  for (int bl = warp; bl < NT; bl += 4) {
+    const int b = n0 + bl;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    float lse2 = -INFINITY;
+    if (b < p.batch) {
+      const int n = clamp_len(__ldg(p.seq_lens + b), cap_len, &err);
+      const int tb = tiles_of(n);
+      if (tb > 0) {
+        const int pb = pref[bl];
+        const int c0 = pb / quota, c1 = (pb + tb - 1) / quota;
+        float mx = -INFINITY;
+        for (int c = c0; c <= c1; ++c) mx = fmaxf(mx, __ldg(p.lse_part + (size_t)(b + c) * p.h + head));
+        float sum = 0.f;
+        for (int c = c0; c <= c1; ++c) sum += exp2f(__ldg(p.lse_part + (size_t)(b + c) * p.h + head) - mx);
+        lse2 = mx + log2f(sum);
+        for (int c = c0; c <= c1; ++c) {
+          const float w = exp2f(__ldg(p.lse_part + (size_t)(b + c) * p.h + head) - lse2);
+          const float* src = p.o_part + ((size_t)(b + c) * p.h + head) * DB + lane * PER;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] += w * __ldg(src + e);
+        }
+      }
+      if (lane == 0 && p.lse_out) p.lse_out[(size_t)b * p.h + head] = tb > 0 ? lse2 * kLn2 : -INFINITY;
+    }
+    if constexpr (LATENT_ONLY) {
+      if (b < p.batch) {
+        float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) dst[e] = acc[e];
+      }
+    } else {
+      // lane's PER features start at byte lane*PER*2 of the row; write in 2/4/8/16-byte pieces
+#pragma unroll
+      for (int e = 0; e < PER; e += 2) {
+        const int f = lane * PER + e;
+        uint8_t* reg = Bo + (f / Sh::BW) * Sh::B4_REG;
+        const uint32_t off = swizzle(bl * Sh::BROWB + (f % Sh::BW) * 2, Sh::BROWB);
+        if constexpr (PER == 1) {
+          *reinterpret_cast<__nv_bfloat16*>(reg + off) = __float2bfloat16_rn(acc[0]);
+        } else {
+          *reinterpret_cast<uint32_t*>(reg + off) = pack_bf16x2(acc[e], acc[e + 1]);
+        }
+      }
+    }
+  }
+  if (err) atomicOr(err_flag, 1);
+
+  if constexpr (!LATENT_ONLY) {
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (warp == 0) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns));
+      if (ok) {
+        tc_fence_after();
+        if (lane == 0) {
+          constexpr uint32_t idesc = idesc_bf16_f32(128, NT, true, false);
+          constexpr int KPR = Sh::BW / 16;
+#pragma unroll
+          for (int ks = 0; ks < DB / 16; ++ks) {
+            const uint64_t a = smem_desc(smem_u32(A + ks * 16 * Sh::AROWB), Sh::A4_LBO, 8 * Sh::AROWB,
+                                         swizzle_code(Sh::AROWB));
+            const uint64_t b = smem_desc(smem_u32(Bo + (ks / KPR) * Sh::B4_REG + (ks % KPR) * 32), 16,
+                                         8 * Sh::BROWB, swizzle_code(Sh::BROWB));
+            umma_bf16(tbase, a, b, idesc, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[1]);
+        }
+        __syncwarp();
+      }
+    }
+    const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
+    if (ok) {
+      tc_fence_after();
+      const int d = warp * 32 + lane;
+      float v[NT];
+      tmem_load_row<NT>(tbase + (static_cast<uint32_t>(warp * 32) << 16), v);
+      tmem_ld_wait();
+      if (d < DH) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const int b = n0 + n;
+          if (b >= p.batch) continue;
+          const size_t o = ((size_t)b * p.h + head) * DH + d;
+          if (p.out_f32)
+            static_cast<float*>(p.out)[o] = v[n];
+          else
+            static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v[n]);
+        }
+      }
+    }
+    if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (*err_flag) set_status(p.status, kErrSeqLen);
+    if (*abort_flag) set_status(p.status, kErrTimeout);
+  }
+  if (!LATENT_ONLY && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Sh::TMEM4);
+  }
+}
+
+}  // namespace mlra
