@@ -1,0 +1,365 @@
+"""Benchmark of one MLRA decode step (query absorption, split-KV latent attention, log-sum-exp
+combine + W^UV up-projection) on the MLRA-4 workload h=128, d_h=128, d_c=512 (4 blocks of
+128), d_r=64, batch 32, context 8192, bf16 paged cache (64-token pages, seeded permutation).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Prints one JSON line. The metric is the latent-cache stream rate of a whole decode step:
+cache bytes of the step / step time (GB/s), with the step time in ms_per_step. Under
+torchrun (N > 1) every rank runs its own replica of the workload (weak scaling; the path
+has no data exchange) and rank 0 reports the total over ranks / the slowest rank's time.
+
+`--impl reference` times the float64 oracle (oracle/) on this host's cores: each step is a
+bounded sample of the same workload (a few (sequence, head) pairs), scaled to the metric by
+the fraction of the workload it covers.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MLRA-4 decode attn: achieved HBM GB/s (% of peak), µs/step at B=32, n=8192"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def cache_bytes(w: W.Workload, seq_lens) -> int:
+    """Algorithmic bytes of the latent-cache stream of one step: each cached token's row
+    [c | k^R] read once (bf16) plus one 4-byte page-table entry per 64 tokens."""
+    toks = int(sum(int(n) for n in seq_lens))
+    pages = int(sum((int(n) + 63) // 64 for n in seq_lens))
+    return toks * (w.d_c + w.d_r) * 2 + pages * 4
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ["common.cuh", "decode.cuh"]:
+        with open(os.path.join(ROOT, "rank_latent_kv_mlra_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch of the decode kernel from a committed ncu summary, if the kernel
+    source has not changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    ent = rec.get("workloads", {}).get(workload_name)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx = float(p[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(impl):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if impl == "ours" else "gloo"
+        if impl == "ours":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# float64 oracle on host cores
+# ---------------------------------------------------------------------------------------
+
+def oracle_sample_rate(w, inp, pairs_per_step, steps, warmup):
+    """Times the oracle as it stands on (sequence, head) pairs of the workload; returns
+    (GB/s-equivalent, seconds per step, threads)."""
+    from oracle import mlra_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    seq_lens = inp["seq_lens"].cpu().numpy()
+    q = inp["q"].double().cpu().numpy()
+    wuk = inp["w_uk"].double().cpu().numpy()
+    wuv = inp["w_uv"].double().cpu().numpy()
+    pt = inp["page_table"].cpu().numpy()
+    rng = np.random.default_rng(0)
+    total_heads = w.batch * w.h
+    full_bytes = cache_bytes(w, seq_lens)
+    sub_pools = {}
+
+    def rows_of(b):
+        if b not in sub_pools:
+            n = int(seq_lens[b])
+            pages = pt[b, :(n + 63) // 64]
+            sp = inp["pool"][torch.as_tensor(pages, device=inp["pool"].device).long()].float().cpu().numpy()
+            sub_pools[b] = O.gather_rows(sp, np.arange(len(pages))[None, :], 0, n)
+        return sub_pools[b]
+
+    def step():
+        for _ in range(pairs_per_step):
+            b = int(rng.integers(0, w.batch))
+            hd = int(rng.integers(0, w.h))
+            O.decode_heads(q[b], wuk, wuv, rows_of(b), [hd], w.k, w.d_r)
+
+    for _ in range(warmup):
+        step()
+    # gathering rows is the oracle's page walk; it is timed too, per sequence first seen
+    sub_pools.clear()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = time.perf_counter() - t0
+    bytes_done = full_bytes * (pairs_per_step * steps) / total_heads
+    return bytes_done / dt / 1e9, dt / steps, threads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_workload(w, device=dev)
+    rate, sec_per_step, threads = oracle_sample_rate(w, inp, 1, args.steps, args.warmup)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
+                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "each step: the float64 oracle on one random (sequence, head) pair "
+                                   f"of the {w.name} workload; value scaled by the fraction of the "
+                                   "workload's heads covered"},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# our CUDA path
+# ---------------------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import rank_latent_kv_mlra_b200 as M
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_workload(w, device=dev)
+    hdl = M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"])
+    B = w.batch
+    out = torch.empty(B, w.h, w.d_h, device=dev, dtype=torch.bfloat16)
+    ws = M.alloc_workspace(hdl, B, dev)
+    stream = torch.cuda.current_stream(dev)
+    args_dec = (hdl, inp["q"], inp["pool"], inp["page_table"], inp["seq_lens"], out)
+    nbytes = cache_bytes(w, inp["seq_lens"].cpu().tolist())
+
+    # correctness guard on this very launch configuration
+    M.mlra_decode(*args_dec, workspace=ws)
+    torch.cuda.synchronize()
+    status = M.mlra_get_status(ws)
+    if status != 0:
+        raise RuntimeError(f"decode status {status}")
+
+    for _ in range(args.warmup):
+        M.mlra_decode(*args_dec, workspace=ws)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        M.mlra_decode(*args_dec, workspace=ws)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+
+    # per-kernel times: events between the three kernels (no programmatic overlap here)
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        M.mlra_decode_profiled(*args_dec, kevs[i], workspace=ws)
+    torch.cuda.synchronize()
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kevs) / args.steps for i in range(3)]
+    clk = clocks.stop()
+
+    # end to end through the public API: pinned host q and seq_lens in, output back to host
+    q_host = inp["q"].cpu().pin_memory()
+    sl_host = inp["seq_lens"].cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_dev = torch.empty_like(inp["q"])
+    sl_dev = torch.empty_like(inp["seq_lens"])
+    e2e_args = (hdl, q_dev, inp["pool"], inp["page_table"], sl_dev, out)
+    for _ in range(max(3, args.warmup // 10)):
+        q_dev.copy_(q_host, non_blocking=True)
+        sl_dev.copy_(sl_host, non_blocking=True)
+        M.mlra_decode(*e2e_args, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_steps = max(10, args.steps // 4)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        q_dev.copy_(q_host, non_blocking=True)
+        sl_dev.copy_(sl_host, non_blocking=True)
+        M.mlra_decode(*e2e_args, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
+    k_ms = [max_over_ranks(x, world, dev) for x in k_ms]
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_hbm_peak()
+    value = world * nbytes / (step_ms_max * 1e-3) / 1e9
+    achieved = nbytes / (k_ms[1] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms_max, "us_per_step": step_ms_max * 1e3,
+        "pct_of_hbm_peak": 100.0 * value / world / peak,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; inputs larger than L2: the 302 MB cache stream evicts the 126 MB L2 each step)",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
+                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
+                   "l2": "inputs larger than L2", "parallelism": f"replicas{world}",
+                   "cache_bytes_per_step": nbytes},
+        "kernels_ms": {"absorb": k_ms[0], "decode": k_ms[1], "combine_uproj": k_ms[2]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "mlra_decode_kernel (split-KV latent attention)",
+                     "traffic": recorded_traffic(w.name)},
+        "e2e": {"value": world * nbytes / (e2e_ms_max * 1e-3) / 1e9, "unit": UNIT,
+                "ms_per_step": e2e_ms_max,
+                "h2d_bytes_per_step": q_host.numel() * q_host.element_size() + sl_host.numel() * 4,
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        pairs = max(1, args.cpu_pairs)
+        rate, sec, threads = oracle_sample_rate(w, inp, pairs, 1, 0)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"float64 oracle on {pairs} random (sequence, head) pairs of "
+                                          f"{w.name} ({sec:.1f} s), scaled by the fraction of the "
+                                          "workload's heads covered"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
+    ap.add_argument("--cpu-pairs", type=int, default=400)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args.impl)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

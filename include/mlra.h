@@ -109,6 +109,16 @@ int mlra_decode_latent(mlra_handle h, const void* q, mlra_dtype q_dtype, const v
                        const int32_t* seq_lens, int batch, float* latent_out, float* lse,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* mlra_decode for profiling: records events[0..3] (cudaEvent_t, created by the caller) on
+ * `stream` before the absorb kernel, between the kernels and after the last one, and
+ * launches without programmatic overlap so each event interval is one kernel's own time.
+ * Results are identical to mlra_decode. */
+int mlra_decode_profiled(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                         int num_pages, const int32_t* page_table, int pt_stride,
+                         const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
+                         float* lse, void* workspace, size_t ws_bytes, void* const* events,
+                         void* stream);
+
 /* Writes new cache rows: token i goes to sequence seq_ids[i] at position positions[i], i.e.
  * slot positions[i] % page_size of page page_table[seq_ids[i]*pt_stride + positions[i]/page_size].
  *   c_new   device [n_tokens][d_c], kr_new device [n_tokens][d_rope], dtype in_dtype;

@@ -34,6 +34,7 @@ STATUS = {
 EXPORTED = [
     "mlra_create", "mlra_destroy", "mlra_workspace_size", "mlra_decode", "mlra_decode_latent",
     "mlra_append_cache", "mlra_plan", "mlra_get_info", "mlra_get_status", "mlra_status_string",
+    "mlra_decode_profiled",
 ]
 
 
@@ -74,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mlra_workspace_size.argtypes = [P, I, ctypes.POINTER(S)]
     lib.mlra_decode.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, S, P]
     lib.mlra_decode_latent.argtypes = [P, P, I, P, I, P, I, P, I, P, P, P, S, P]
+    lib.mlra_decode_profiled.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, S, P, P]
     lib.mlra_append_cache.argtypes = [P, P, I, P, I, I, P, P, P, P, I, I, P, P]
     lib.mlra_plan.argtypes = [P, P, I, I, P, I, P, P]
     lib.mlra_get_info.argtypes = [P, ctypes.POINTER(mlra_info)]
@@ -191,6 +193,23 @@ def mlra_decode(handle: Handle, q, pool, page_table, seq_lens, out, lse=None, wo
         handle.ptr, _ptr(q), _dtype(q), _ptr(pool), pool.shape[0], _ptr(page_table),
         page_table.shape[1], _ptr(seq_lens), B, _ptr(out), _dtype(out), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream(stream)), "mlra_decode")
+    return workspace
+
+
+def mlra_decode_profiled(handle: Handle, q, pool, page_table, seq_lens, out, events, lse=None,
+                         workspace=None, stream=None):
+    """mlra_decode that records four torch.cuda.Event objects around its three kernels."""
+    if workspace is None:
+        workspace = alloc_workspace(handle, q.shape[0], q.device)
+    B = _decode_common(handle, q, pool, page_table, seq_lens, workspace)
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the CUDA event on its first record
+            e.record(stream or torch.cuda.current_stream())
+    ev = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+    _check(load_library().mlra_decode_profiled(
+        handle.ptr, _ptr(q), _dtype(q), _ptr(pool), pool.shape[0], _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, _ptr(out), _dtype(out), _ptr(lse), _ptr(workspace),
+        workspace.numel(), ev, _stream(stream)), "mlra_decode_profiled")
     return workspace
 
 

@@ -124,6 +124,10 @@ cudaError_t prep_proj_all() {
   return prep_proj<DB, DH, 128>();
 }
 
+// Programmatic dependent launch is on except inside a profiled call (thread-local, so a
+// profiled call on one thread does not change another thread's launches).
+thread_local bool g_use_pdl = true;
+
 // `attr` must outlive the launch call that uses the returned config.
 cudaLaunchConfig_t launch_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
                               cudaLaunchAttribute* attr) {
@@ -132,7 +136,7 @@ cudaLaunchConfig_t launch_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s
   c.blockDim = block;
   c.dynamicSmemBytes = smem;
   c.stream = s;
-  if (pdl) {
+  if (pdl && g_use_pdl) {
     attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr->val.programmaticStreamSerializationAllowed = 1;
     c.attrs = attr;
@@ -215,7 +219,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
                const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch, void* out,
                mlra_dtype out_dtype, float* lse, float* latent_out, void* workspace, size_t ws_bytes,
-               void* stream, int inject_stall, unsigned long long wait_limit_ns) {
+               void* stream, int inject_stall, unsigned long long wait_limit_ns,
+               void* const* events = nullptr) {
   if (!h || !q || !pool || !page_table || !seq_lens || !workspace) return MLRA_ERR_INVALID_ARG;
   if (!out && !latent_out) return MLRA_ERR_INVALID_ARG;
   if (batch <= 0 || batch > 4096 || num_pages <= 0 || pt_stride <= 0) return MLRA_ERR_INVALID_ARG;
@@ -285,25 +290,39 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
 
   cudaError_t e = cudaSuccess;
   const bool latent = latent_out != nullptr;
+  // profiling: events between the kernels (and no programmatic overlap, so each interval
+  // is one kernel's own time)
+  const bool prof = events != nullptr;
+  auto rec = [&](int i) {
+    if (prof && e == cudaSuccess) e = cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+  };
+  g_use_pdl = !prof;
+  rec(0);
   switch (h->var) {
     case kTiny:
       e = dispatch_absorb<32, 32>(h, pp, batch, s);
+      rec(1);
       if (e == cudaSuccess) e = launch_decode<DecTiny>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
       if (e == cudaSuccess)
         e = latent ? dispatch_uproj<32, 32, true>(h, pp, batch, s) : dispatch_uproj<32, 32, false>(h, pp, batch, s);
       break;
     case kMlra4:
       e = dispatch_absorb<128, 128>(h, pp, batch, s);
+      rec(1);
       if (e == cudaSuccess)
         e = h->stages == 3 ? launch_decode<DecMlra4q2>(h, mc, mr, mqc, mqr, dp, s)
                            : launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
       if (e == cudaSuccess)
         e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
                    : dispatch_uproj<128, 128, false>(h, pp, batch, s);
       break;
     case kMlra2:
       e = dispatch_absorb<256, 128>(h, pp, batch, s);
+      rec(1);
       if (e == cudaSuccess) e = launch_decode<DecMlra2>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
       if (e == cudaSuccess)
         e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
                    : dispatch_uproj<256, 128, false>(h, pp, batch, s);
@@ -311,6 +330,8 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
     default:
       return MLRA_ERR_UNSUPPORTED;
   }
+  rec(3);
+  g_use_pdl = true;
   return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
 }
 
@@ -473,6 +494,18 @@ const char* mlra_status_string(int code) {
     case MLRA_ERR_SEQ_LEN: return "sequence length outside its page-table row";
     default: return "unknown status";
   }
+}
+
+int mlra_decode_profiled(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                         int num_pages, const int32_t* page_table, int pt_stride,
+                         const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
+                         float* lse, void* workspace, size_t ws_bytes, void* const* events,
+                         void* stream) {
+  if (!out || !events) return MLRA_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (!events[i]) return MLRA_ERR_INVALID_ARG;
+  return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, out_dtype,
+                    lse, nullptr, workspace, ws_bytes, stream, 0, kWaitLimitNs, events);
 }
 
 // Test hook (not in the public header): a decode whose producer withholds its first tile, so
