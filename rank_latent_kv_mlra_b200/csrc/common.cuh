@@ -31,6 +31,24 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// Timeline trace points. They compile to nothing unless MLRA_TRACE is defined (a profiling
+// build); then point `id` of kernel `k` in this CTA records %globaltimer into g_mlra_trace.
+#ifdef MLRA_TRACE
+__device__ unsigned long long* g_mlra_trace;
+constexpr int kTracePoints = 256;
+#define MLRA_TRACE_POINT(k, id)                                                              \
+  do {                                                                                       \
+    const unsigned long long ts_ = global_timer_ns();                                        \
+    if (g_mlra_trace != nullptr && (id) < kTracePoints)                                      \
+      g_mlra_trace[((size_t)(k) * 1024 + blockIdx.x + blockIdx.y * gridDim.x) * kTracePoints + \
+                   (id)] = ts_;                                                              \
+  } while (0)
+#else
+#define MLRA_TRACE_POINT(k, id) \
+  do {                          \
+  } while (0)
+#endif
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 // ------------------------------------------------------------------------------------
@@ -67,6 +85,19 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test (never suspends the thread), for polling several barriers in turn.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -245,11 +276,28 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-// Loads / stores N (16, 32 or 64) consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// Loads / stores N (8, 16, 32 or 64) consecutive fp32 columns of this thread's TMEM lane.
 template <int N>
 __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&v)[N]) {
-  static_assert(N == 16 || N % 32 == 0, "row width");
-  if constexpr (N == 16) {
+  static_assert(N == 8 || N == 16 || N % 32 == 0, "row width");
+  if constexpr (N == 8) {
+    uint32_t r[8];
+    tmem_ld8(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+  } else if constexpr (N == 16) {
     uint32_t r[16];
     tmem_ld16(taddr, r);
 #pragma unroll
@@ -266,7 +314,12 @@ __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&v)[N]) {
 }
 template <int N>
 __device__ __forceinline__ void tmem_store_row(uint32_t taddr, const float (&v)[N]) {
-  if constexpr (N == 16) {
+  if constexpr (N == 8) {
+    uint32_t r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __float_as_uint(v[i]);
+    tmem_st8(taddr, r);
+  } else if constexpr (N == 16) {
     uint32_t r[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(v[i]);

@@ -15,8 +15,9 @@
 // Tokens sit on the MMA's M dimension because a block serves only h/k heads (32 for MLRA-4),
 // fewer than the 64/128 rows an MMA needs.
 //
-// Roles (192 threads): warp 0 issues TMA loads of pages and queries, warp 1 allocates TMEM
-// and issues the MMAs, warps 2..5 run the softmax and write the partial results. They
+// Roles (64 + 128*NWG threads): warp 0 issues TMA loads of pages and queries, warp 1
+// allocates TMEM and issues the MMAs, warps 2.. form NWG softmax warpgroups (each owns a
+// slice of the heads) that run the softmax and write the partial results. They
 // hand off through mbarriers; each wait is bounded (see mbar_wait).
 //
 // Softmax detail: each thread owns one token row of S^T and all its heads. The running
@@ -39,6 +40,9 @@ struct DecodeShape {
   static constexpr int DB = DB_;      // latent block width d_c / k
   static constexpr int DR = DR_;      // RoPE key width
   static constexpr int NP = NP_;      // heads per CTA (MMA N), 16 / 32 / 64
+  static constexpr int NWG = 2;       // softmax warpgroups; each owns NP / NWG heads
+  static constexpr int HW = NP / NWG;
+  static constexpr int THREADS = 64 + 128 * NWG;
   static constexpr int STAGES = STAGES_;
   static constexpr int QBUF = QBUF_;  // query buffers
   static constexpr int PBUF = PBUF_;  // probability buffers
@@ -103,15 +107,15 @@ struct DecodeParams {
   int inject_stall;  // test hook: the producer withholds its first tile
 };
 
-// Reduce NP values across the 32 lanes of a warp and scatter the results: afterwards lane l
-// holds in v[0..max(1, NP/32)) the reduction of heads [l*NP/32, (l+1)*NP/32) (NP >= 32) or of
-// head (l & 15) (NP == 16).
+// Reduce N per-head values across the 32 lanes of a warp and scatter the results: afterwards
+// lane l holds in v[0..max(1, N/32)) the reduction over all lanes of heads
+// [l*N/32, (l+1)*N/32) when N >= 32, or of head (l mod N) when N < 32.
 template <bool IS_MAX>
 __device__ __forceinline__ float red_op(float a, float b) {
   return IS_MAX ? fmaxf(a, b) : a + b;
 }
-template <int OFF, int N, bool IS_MAX, int NP>
-__device__ __forceinline__ void rs_step(float (&v)[NP], int lane) {
+template <int OFF, int N, bool IS_MAX, int L>
+__device__ __forceinline__ void rs_step(float (&v)[L], int lane) {
   const bool upper = (lane & OFF) != 0;
 #pragma unroll
   for (int x = 0; x < N / 2; ++x) {
@@ -120,36 +124,60 @@ __device__ __forceinline__ void rs_step(float (&v)[NP], int lane) {
     v[x] = red_op<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, OFF));
   }
 }
-template <int NP, bool IS_MAX>
-__device__ __forceinline__ void warp_reduce_scatter(float (&v)[NP], int lane) {
-  if constexpr (NP == 16) {
+template <int OFF, int N, bool IS_MAX, int L>
+__device__ __forceinline__ void rs_chain(float (&v)[L], int lane) {
+  if constexpr (OFF >= 1 && N >= 2) {
+    rs_step<OFF, N, IS_MAX>(v, lane);
+    rs_chain<OFF / 2, N / 2, IS_MAX>(v, lane);
+  }
+}
+template <int OFF, int N, bool IS_MAX, int L>
+__device__ __forceinline__ void plain_chain(float (&v)[L]) {
+  if constexpr (OFF >= N) {
 #pragma unroll
-    for (int x = 0; x < 16; ++x) v[x] = red_op<IS_MAX>(v[x], __shfl_xor_sync(0xffffffffu, v[x], 16));
-    rs_step<8, 16, IS_MAX>(v, lane);
-    rs_step<4, 8, IS_MAX>(v, lane);
-    rs_step<2, 4, IS_MAX>(v, lane);
-    rs_step<1, 2, IS_MAX>(v, lane);
+    for (int x = 0; x < N; ++x) v[x] = red_op<IS_MAX>(v[x], __shfl_xor_sync(0xffffffffu, v[x], OFF));
+    plain_chain<OFF / 2, N, IS_MAX>(v);
+  }
+}
+template <int N, bool IS_MAX>
+__device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
+  if constexpr (N >= 32) {
+    rs_chain<16, N, IS_MAX>(v, lane);
   } else {
-    rs_step<16, NP, IS_MAX>(v, lane);
-    rs_step<8, NP / 2, IS_MAX>(v, lane);
-    rs_step<4, NP / 4, IS_MAX>(v, lane);
-    rs_step<2, NP / 8, IS_MAX>(v, lane);
-    rs_step<1, NP / 16, IS_MAX>(v, lane);
+    plain_chain<16, N, IS_MAX>(v);  // fold lanes that differ above bit log2(N)
+    rs_chain<N / 2, N, IS_MAX>(v, lane);
   }
 }
 // Writes the scattered per-head values of this lane to dst[h].
-template <int NP>
-__device__ __forceinline__ void store_scattered(const float (&v)[NP], float* dst, int lane) {
-  if constexpr (NP == 16) {
-    if (lane < 16) dst[lane] = v[0];
+template <int N>
+__device__ __forceinline__ void store_scattered(const float (&v)[N], float* dst, int lane) {
+  if constexpr (N < 32) {
+    if (lane < N) dst[lane] = v[0];
   } else {
 #pragma unroll
-    for (int x = 0; x < NP / 32; ++x) dst[lane * (NP / 32) + x] = v[x];
+    for (int x = 0; x < N / 32; ++x) dst[lane * (N / 32) + x] = v[x];
   }
 }
 
+// Pairwise fp32 ops on the packed f32x2 datapath.
+__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
+  return (static_cast<unsigned long long>(__float_as_uint(b)) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ void sub_f32x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2pack(a0, a1)), "l"(f2pack(b0, b1)));
+  d0 = __uint_as_float(static_cast<uint32_t>(d));
+  d1 = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+__device__ __forceinline__ void add_f32x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2pack(a0, a1)), "l"(f2pack(b0, b1)));
+  d0 = __uint_as_float(static_cast<uint32_t>(d));
+  d1 = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+
 template <class Sh>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Sh::THREADS, 1)
     mlra_decode_kernel(const __grid_constant__ CUtensorMap map_c,
                        const __grid_constant__ CUtensorMap map_r,
                        const __grid_constant__ CUtensorMap map_qc,
@@ -161,7 +189,6 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* stages = smem + Sh::OFF_STAGES;
   uint8_t* qbufs = smem + Sh::OFF_Q;
   uint8_t* pbufs = smem + Sh::OFF_P;
-  float* m_sm = reinterpret_cast<float*>(smem + Sh::OFF_M);
   float* red_sm = reinterpret_cast<float*>(smem + Sh::OFF_RED);
   Segment* segs = reinterpret_cast<Segment*>(smem + Sh::OFF_SEG);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::OFF_BAR);
@@ -188,6 +215,7 @@ __global__ void __launch_bounds__(192, 1)
   const int head0 = blk * p.heads_block + chunk * NP;
   const int nheads = min(NP, p.heads_block - chunk * NP);
   const int cap_len = p.pt_stride * kPage;
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -200,8 +228,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sfull_bar[s], 1);
-      mbar_init(&sfree_bar[s], 4);
-      mbar_init(&pfull_bar[s], 4);
+      mbar_init(&sfree_bar[s], 4 * Sh::NWG);
+      mbar_init(&pfull_bar[s], 4 * Sh::NWG);
       mbar_init(&pvdone_bar[s], 1);
     }
     mbar_init(mmadone_bar, 1);
@@ -223,6 +251,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 1);
 
   // ---- plan: which flattened tiles this group owns (seq_lens do not depend on the
   // previous kernel, so this overlaps its tail under programmatic dependent launch) ----
@@ -236,15 +265,12 @@ __global__ void __launch_bounds__(192, 1)
   // pipeline counters persist across segment-list refills
   uint32_t it = 0;      // tiles consumed/produced so far by this role
   uint32_t segc = 0;    // segments so far
-  // MMA-role state of the previous tile (its PV is issued one tile late)
-  bool prev_valid = false, prev_first = false;
-  uint32_t prev_it = 0;
   // producer: last issued phase per stage, for the drain at the end
   uint32_t issued_mask = 0;
-  // softmax-role partial sums
-  float l_part[NP];
+  // softmax-role partial sums (the warpgroup's heads)
+  float l_part[Sh::HW];
 #pragma unroll
-  for (int x = 0; x < NP; ++x) l_part[x] = 0.f;
+  for (int x = 0; x < Sh::HW; ++x) l_part[x] = 0.f;
 
   int b_start = 0, p_start = 0;
   bool more = lo < hi;
@@ -255,12 +281,14 @@ __global__ void __launch_bounds__(192, 1)
     more = more_i != 0;
     b_start = rb;
     p_start = rp;
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 2);
 
     if (warp == 0) {
       // ============================== TMA producer ==============================
       const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
       grid_dependency_wait();  // q_pack and the reset status word come from the absorb kernel
+      if (lane == 0) MLRA_TRACE_POINT(1, 3);
       if (lane == 0 && *plan_err) set_status(p.status, kErrSeqLen);
       for (int si = 0; si < nseg && !*abort_flag; ++si) {
         const Segment sg = segs[si];
@@ -282,17 +310,32 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         ++segc;
-        int pbase = -64, pid = 0;
+        // Page ids of this segment, a 64-page window held two registers per lane; the loads
+        // for the upper half are issued 16 tiles before they are needed, so the producer
+        // never waits on a page-table read.
+        const int* pt_row = p.page_table + (size_t)sg.b * p.pt_stride;
+        int wb = 2 * sg.tile_begin;
+        auto load_ids = [&](int base) {
+          const int pp = base + lane;
+          return pp < pages_b ? __ldg(pt_row + pp) : 0;
+        };
+        int w0 = load_ids(wb), w1 = load_ids(wb + 32);
+        auto page_id = [&](int pg) {  // warp-uniform pg in [wb, wb + 64); only the half
+                                       // that holds pg is read, so a fresh load of the other
+                                       // half is not waited for
+          if (pg - wb < 32) return __shfl_sync(0xffffffffu, w0, pg - wb);
+          return __shfl_sync(0xffffffffu, w1, pg - wb - 32);
+        };
         for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++it) {
           const int p0 = 2 * t;
-          if (p0 + 1 >= pbase + 32) {
-            pbase = p0;
-            const int pp = pbase + lane;
-            pid = pp < pages_b ? __ldg(p.page_table + (size_t)sg.b * p.pt_stride + pp) : 0;
+          if (p0 >= wb + 32) {  // slide the window by 32 pages
+            wb += 32;
+            w0 = w1;
+            w1 = load_ids(wb + 32);
           }
-          int id0 = __shfl_sync(0xffffffffu, pid, p0 - pbase);
-          int id1 = __shfl_sync(0xffffffffu, pid, p0 + 1 - pbase);
+          int id0 = page_id(p0);
           const int npg = (p0 + 1 < pages_b) ? 2 : 1;
+          int id1 = page_id(min(p0 + 1, pages_b - 1));
           ok = true;
           if (lane == 0) {
             if (id0 < 0 || id0 >= p.num_pages) { set_status(p.status, kErrPageOob); id0 = 0; }
@@ -300,6 +343,7 @@ __global__ void __launch_bounds__(192, 1)
             const int st = it % STAGES;
             ok = mbar_wait(&empty_bar[st], ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns);
             if (ok && !(p.inject_stall && it == 0)) {
+              MLRA_TRACE_POINT(1, 8 + min((int)it, 31));
               uint8_t* dst = stages + st * Sh::STAGE_BYTES;
               mbar_arrive_expect_tx(&full_bar[st], npg * Sh::PAGE_TX);
               issued_mask |= 1u << st;
@@ -319,99 +363,150 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else if (warp == 1) {
       // ============================== MMA issuer ==============================
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NP, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NP, true, true);
-      auto issue_pv = [&](uint32_t j, bool first) -> bool {
-        bool ok = mbar_wait(&pfull_bar[j & 1], (j >> 1) & 1, abort_flag, p.wait_limit_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) return false;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t st_addr = smem_u32(stages + (j % STAGES) * Sh::STAGE_BYTES);
-          const uint32_t p_addr = smem_u32(pbufs + (j % Sh::PBUF) * Sh::P_BYTES);
-#pragma unroll
-          for (int mt = 0; mt < Sh::NMT; ++mt) {
-#pragma unroll
-            for (int ks = 0; ks < kTile / 16; ++ks) {
-              const uint64_t a = smem_desc(st_addr + mt * (128 / Sh::CW) * Sh::C_REG + ks * 16 * Sh::C_ROWB,
-                                           Sh::PV_LBO, 8 * Sh::C_ROWB, swizzle_code(Sh::C_ROWB));
-              const uint64_t b = smem_desc(p_addr + ks * 16 * Sh::P_ROWB, Sh::P_BYTES,
-                                           8 * Sh::P_ROWB, swizzle_code(Sh::P_ROWB));
-              umma_bf16(tbase + Sh::O_COL + mt * NP, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
-            }
+      // One thread issues. Two cursors walk the list's tiles: QK(i) needs tile i's pages
+      // (and, at a segment start, its query) plus a free S buffer; PV(i) needs P(i) from the
+      // softmax. Whichever is ready goes first, PV preferred: it releases a pipeline stage, so
+      // late page data never holds back a finished tile's PV and with it the next loads.
+      // Polling never suspends the thread, so neither condition waits behind the other.
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NP, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NP, true, true);
+        struct Cursor {
+          int si, t;
+          uint32_t it, segc;
+        };
+        Cursor cq{0, nseg > 0 ? segs[0].tile_begin : 0, it, segc};
+        Cursor cp = cq;
+        uint32_t list_tiles = 0;
+        for (int i = 0; i < nseg; ++i) list_tiles += segs[i].tile_end - segs[i].tile_begin;
+        const uint32_t it_end = it + list_tiles;
+        auto advance = [&](Cursor& c) {
+          ++c.it;
+          if (++c.t == segs[c.si].tile_end) {
+            ++c.si;
+            ++c.segc;
+            if (c.si < nseg) c.t = segs[c.si].tile_begin;
           }
-          umma_commit(&empty_bar[j % STAGES]);
-          umma_commit(&pvdone_bar[j & 1]);
-        }
-        __syncwarp();
-        return true;
-      };
-      bool ok = true;
-      for (int si = 0; si < nseg && ok; ++si) {
-        const Segment sg = segs[si];
-        const int qb = segc % Sh::QBUF;
-        ok = __all_sync(0xffffffffu, mbar_wait(&qfull_bar[qb], (segc / Sh::QBUF) & 1, abort_flag,
-                                               p.wait_limit_ns));
-        if (!ok) break;
-        const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
-        for (int t = sg.tile_begin; t < sg.tile_end && ok; ++t, ++it) {
-          const int st = it % STAGES;
-          ok = mbar_wait(&full_bar[st], (it / STAGES) & 1, abort_flag, p.wait_limit_ns);
-          if (ok && it >= 2)
-            ok = mbar_wait(&sfree_bar[it & 1], ((it >> 1) - 1) & 1, abort_flag, p.wait_limit_ns);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t st_addr = smem_u32(stages + st * Sh::STAGE_BYTES);
-            const uint32_t d = tbase + Sh::S_COL0 + (it & 1) * NP;
-            uint32_t acc = 0;
+        };
+        bool q_ready = false;  // query of cq's segment has landed
+        uint64_t t_idle = 0;
+#ifdef MLRA_TRACE
+        uint32_t traced_arrival = 0xffffffffu;
+#endif
+        while (cp.it < it_end) {
+          bool issued = false;
+          if (cp.it < cq.it && mbar_poll(&pfull_bar[cp.it & 1], (cp.it >> 1) & 1)) {
+            // ---- PV(cp.it): O^T += C^T P^T
+            tc_fence_after();
+            MLRA_TRACE_POINT(1, 72 + min((int)cp.it, 31));
+            const bool first = cp.t == segs[cp.si].tile_begin;
+            const uint32_t st_addr = smem_u32(stages + (cp.it % STAGES) * Sh::STAGE_BYTES);
+            const uint32_t p_addr = smem_u32(pbufs + (cp.it % Sh::PBUF) * Sh::P_BYTES);
 #pragma unroll
-            for (int r = 0; r < Sh::NC; ++r) {
+            for (int mt = 0; mt < Sh::NMT; ++mt) {
 #pragma unroll
-              for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
-                const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                             swizzle_code(Sh::C_ROWB));
-                const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                             swizzle_code(Sh::C_ROWB));
-                umma_bf16(d, a, b, idesc_qk, acc);
-                acc = 1;
+              for (int ks = 0; ks < kTile / 16; ++ks) {
+                const uint64_t a = smem_desc(st_addr + mt * (128 / Sh::CW) * Sh::C_REG + ks * 16 * Sh::C_ROWB,
+                                             Sh::PV_LBO, 8 * Sh::C_ROWB, swizzle_code(Sh::C_ROWB));
+                const uint64_t b = smem_desc(p_addr + ks * 16 * Sh::P_ROWB, Sh::P_BYTES, 8 * Sh::P_ROWB,
+                                             swizzle_code(Sh::P_ROWB));
+                umma_bf16(tbase + Sh::O_COL + mt * NP, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
               }
             }
-#pragma unroll
-            for (int r = 0; r < Sh::NR; ++r) {
-#pragma unroll
-              for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
-                const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
-                                             8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32,
-                                             16, 8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                umma_bf16(d, a, b, idesc_qk, 1);
-              }
+            umma_commit(&empty_bar[cp.it % STAGES]);
+            umma_commit(&pvdone_bar[cp.it & 1]);
+            advance(cp);
+            issued = true;
+          } else if (cq.it < it_end) {
+            const int qb = cq.segc % Sh::QBUF;
+            const bool seg_first = cq.t == segs[cq.si].tile_begin;
+            if (seg_first && !q_ready) q_ready = mbar_poll(&qfull_bar[qb], (cq.segc / Sh::QBUF) & 1);
+            const bool data = mbar_poll(&full_bar[cq.it % STAGES], (cq.it / STAGES) & 1);
+#ifdef MLRA_TRACE
+            if (data && cq.it != traced_arrival) {
+              traced_arrival = cq.it;
+              MLRA_TRACE_POINT(1, 232 + min((int)cq.it, 23));
             }
-            umma_commit(&sfull_bar[it & 1]);
-            if (t == sg.tile_end - 1) umma_commit(&qempty_bar[qb]);
+#endif
+            if ((!seg_first || q_ready) && data &&
+                (cq.it < 2 || mbar_poll(&sfree_bar[cq.it & 1], ((cq.it >> 1) - 1) & 1))) {
+              // ---- QK(cq.it): S^T = [c_j | k^R] [q~ | q^R]^T
+              tc_fence_after();
+              MLRA_TRACE_POINT(1, 40 + min((int)cq.it, 31));
+              const uint32_t st_addr = smem_u32(stages + (cq.it % STAGES) * Sh::STAGE_BYTES);
+              const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
+              const uint32_t d = tbase + Sh::S_COL0 + (cq.it & 1) * NP;
+              uint32_t acc = 0;
+#pragma unroll
+              for (int r = 0; r < Sh::NC; ++r) {
+#pragma unroll
+                for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
+                  const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                               swizzle_code(Sh::C_ROWB));
+                  const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                               swizzle_code(Sh::C_ROWB));
+                  umma_bf16(d, a, b, idesc_qk, acc);
+                  acc = 1;
+                }
+              }
+#pragma unroll
+              for (int r = 0; r < Sh::NR; ++r) {
+#pragma unroll
+                for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
+                  const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
+                                               8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                  const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
+                                               8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                  umma_bf16(d, a, b, idesc_qk, 1);
+                }
+              }
+              umma_commit(&sfull_bar[cq.it & 1]);
+              if (cq.t == segs[cq.si].tile_end - 1) {
+                umma_commit(&qempty_bar[qb]);
+                q_ready = false;
+              }
+              advance(cq);
+              issued = true;
+            }
           }
-          __syncwarp();
-          if (prev_valid) ok = issue_pv(prev_it, prev_first);
-          prev_valid = true;
-          prev_it = it;
-          prev_first = (t == sg.tile_begin);
+          if (issued) {
+            t_idle = 0;
+          } else {
+            // nothing ready: bounded wait, like every other wait in this kernel
+            if (*abort_flag) break;
+            const uint64_t now = global_timer_ns();
+            if (t_idle == 0) {
+              t_idle = now;
+            } else if (now - t_idle > p.wait_limit_ns) {
+              *abort_flag = 1;
+              break;
+            }
+          }
         }
-        ++segc;
+        it = it_end;
+        segc = cq.segc;
       }
-      // the list's last PV (every list ends on a segment boundary)
-      if (ok && prev_valid) issue_pv(prev_it, prev_first);
-      prev_valid = false;
+      __syncwarp();
+      it = __shfl_sync(0xffffffffu, it, 0);
+      segc = __shfl_sync(0xffffffffu, segc, 0);
     } else {
       // ============================== softmax / epilogue ==============================
-      // The four warps take every decision together: a failed wait in any of them is
-      // folded into a 128-thread OR barrier before anyone leaves, so no warp is left
-      // waiting on a named barrier the others never reach.
-      const int sw = warp - 2;         // 0..3
-      const int q4 = warp & 3;         // TMEM lane quadrant this warp may access
-      const int row = q4 * 32 + lane;  // token row of S^T, feature row of O^T
+      // NWG warpgroups, each owning HW of the CTA's heads (S^T / O^T columns and P bytes of
+      // its own). Within a warpgroup the four warps take every decision together: a failed
+      // wait in any of them is folded into a 128-thread OR barrier before anyone leaves, so no
+      // warp is left waiting on a named barrier the others never reach.
+      constexpr int HW = Sh::HW;
+      const int g = (warp - 2) >> 2;      // warpgroup
+      const int sw = (warp - 2) & 3;      // warp within the group
+      const int q4 = warp & 3;            // TMEM lane quadrant this warp may access
+      const int row = q4 * 32 + lane;     // token row of S^T, feature row of O^T
+      const int hcol = g * HW;            // first head column of this warpgroup
+      const int bar_or = 1 + 2 * g, bar_sync = 2 + 2 * g;
       const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+      float* red = red_sm + g * 4 * HW;
+      float m[HW];                        // running max per head (same in every thread)
+#pragma unroll
+      for (int x = 0; x < HW; ++x) m[x] = -INFINITY;
       bool ok = true;
       for (int si = 0; si < nseg && ok; ++si) {
         const Segment sg = segs[si];
@@ -419,91 +514,100 @@ __global__ void __launch_bounds__(192, 1)
         for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++it) {
           const bool first = (t == sg.tile_begin);
           const bool last = (t == sg.tile_end - 1);
+          const bool tile_full = (t + 1) * kTile <= sg.n;
           const bool valid = t * kTile + row < sg.n;
           bool okl = mbar_wait(&sfull_bar[it & 1], (it >> 1) & 1, abort_flag, p.wait_limit_ns);
           if (it >= Sh::PBUF) {  // the PV that last read this P buffer must be done
             const uint32_t j = it - Sh::PBUF;
             okl = okl && mbar_wait(&pvdone_bar[j & 1], (j >> 1) & 1, abort_flag, p.wait_limit_ns);
           }
+          if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 104 + min((int)it, 31));
           tc_fence_after();
-          float s[NP];
-          tmem_load_row<NP>(tbase + lane_base + Sh::S_COL0 + (it & 1) * NP, s);
+          float s[HW];
+          tmem_load_row<HW>(tbase + lane_base + Sh::S_COL0 + (it & 1) * NP + hcol, s);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sfree_bar[it & 1]);
 
-          float m[NP];
+          if (first) {
 #pragma unroll
-          for (int x = 0; x < NP; ++x) m[x] = first ? -INFINITY : m_sm[x];
-          float dmax = -INFINITY;
-          if (valid) {
-#pragma unroll
-            for (int x = 0; x < NP; ++x) dmax = fmaxf(dmax, s[x] - m[x]);
+            for (int x = 0; x < HW; ++x) m[x] = -INFINITY;
           }
-          const bool need = named_bar_or(1, 128, !okl || first || dmax > kRescaleSlack);
+          // common case: scores relative to the running max, exp2 issued before the vote
+          float xs[HW];
+#pragma unroll
+          for (int x = 0; x < HW; x += 2) sub_f32x2(xs[x], xs[x + 1], s[x], s[x + 1], m[x], m[x + 1]);
+          if (!tile_full && !valid) {
+#pragma unroll
+            for (int x = 0; x < HW; ++x) xs[x] = -INFINITY;
+          }
+          float dm[HW];
+#pragma unroll
+          for (int x = 0; x < HW; ++x) dm[x] = xs[x];
+#pragma unroll
+          for (int w2 = HW / 2; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int x = 0; x < w2; ++x) dm[x] = fmaxf(dm[x], dm[x + w2]);
+          float pr[HW];
+#pragma unroll
+          for (int x = 0; x < HW; ++x) pr[x] = fast_exp2(xs[x]);
+
+          const bool need = named_bar_or(bar_or, 128, !okl || first || dm[0] > kRescaleSlack);
           if (need) {
-            if (named_bar_or(1, 128, !okl || *abort_flag)) { ok = false; break; }
-            float tmax[NP];
+            if (named_bar_or(bar_or, 128, !okl || *abort_flag)) { ok = false; break; }
+            float tmax[HW];
 #pragma unroll
-            for (int x = 0; x < NP; ++x) tmax[x] = valid ? s[x] : -INFINITY;
-            warp_reduce_scatter<NP, true>(tmax, lane);
-            store_scattered<NP>(tmax, red_sm + q4 * NP, lane);
-            named_bar_sync(2, 128);
-            float alpha[NP];
+            for (int x = 0; x < HW; ++x) tmax[x] = valid ? s[x] : -INFINITY;
+            warp_reduce_scatter<HW, true>(tmax, lane);
+            store_scattered<HW>(tmax, red + q4 * HW, lane);
+            named_bar_sync(bar_sync, 128);
+            float alpha[HW];
 #pragma unroll
-            for (int x = 0; x < NP; ++x) {
-              const float tm = fmaxf(fmaxf(red_sm[x], red_sm[NP + x]),
-                                     fmaxf(red_sm[2 * NP + x], red_sm[3 * NP + x]));
+            for (int x = 0; x < HW; ++x) {
+              const float tm = fmaxf(fmaxf(red[x], red[HW + x]), fmaxf(red[2 * HW + x], red[3 * HW + x]));
               const float mn = fmaxf(m[x], tm);
               alpha[x] = first ? 0.f : fast_exp2(m[x] - mn);
               m[x] = mn;
             }
 #pragma unroll
-            for (int x = 0; x < NP; ++x) l_part[x] = first ? 0.f : l_part[x] * alpha[x];
+            for (int x = 0; x < HW; ++x) l_part[x] = first ? 0.f : l_part[x] * alpha[x];
             if (!first) {
               // O holds the sums up to tile it-1: wait for that PV, then rescale its columns
               const bool okr = mbar_wait(&pvdone_bar[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag,
                                          p.wait_limit_ns);
-              if (named_bar_or(1, 128, !okr)) { ok = false; break; }
+              if (named_bar_or(bar_or, 128, !okr)) { ok = false; break; }
               tc_fence_after();
 #pragma unroll
               for (int mt = 0; mt < Sh::NMT; ++mt) {
-                float o[NP];
-                const uint32_t oa = tbase + lane_base + Sh::O_COL + mt * NP;
-                tmem_load_row<NP>(oa, o);
+                float o[HW];
+                const uint32_t oa = tbase + lane_base + Sh::O_COL + mt * NP + hcol;
+                tmem_load_row<HW>(oa, o);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < NP; ++x) o[x] *= alpha[x];
-                tmem_store_row<NP>(oa, o);
+                for (int x = 0; x < HW; ++x) o[x] *= alpha[x];
+                tmem_store_row<HW>(oa, o);
               }
               tmem_st_wait();
             }
-            named_bar_sync(2, 128);  // everyone has read red_sm and the old m_sm
-            if (sw == 0) {
+            named_bar_sync(bar_sync, 128);  // everyone has read red
 #pragma unroll
-              for (int x = 0; x < NP; ++x)
-                if (x % 32 == lane) m_sm[x] = m[x];
-            }
+            for (int x = 0; x < HW; ++x) pr[x] = valid ? fast_exp2(s[x] - m[x]) : 0.f;
           }
+#pragma unroll
+          for (int x = 0; x < HW; x += 2)
+            add_f32x2(l_part[x], l_part[x + 1], l_part[x], l_part[x + 1], pr[x], pr[x + 1]);
           uint8_t* pbuf = pbufs + (it % Sh::PBUF) * Sh::P_BYTES;
 #pragma unroll
-          for (int c = 0; c < Sh::P_ROWB / 16; ++c) {
-            float pv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int x = 8 * c + e;
-              pv[e] = valid ? fast_exp2(s[x] - m[x]) : 0.f;
-              l_part[x] += pv[e];
-            }
+          for (int c = 0; c < HW / 8; ++c) {
             uint4 w;
-            w.x = pack_bf16x2(pv[0], pv[1]);
-            w.y = pack_bf16x2(pv[2], pv[3]);
-            w.z = pack_bf16x2(pv[4], pv[5]);
-            w.w = pack_bf16x2(pv[6], pv[7]);
-            *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + c * 16, Sh::P_ROWB)) = w;
+            w.x = pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]);
+            w.y = pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]);
+            w.z = pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]);
+            w.w = pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]);
+            *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + hcol * 2 + c * 16, Sh::P_ROWB)) = w;
           }
-          if (last && !valid) {
+          if (g == 0 && last && !valid) {
             // rows past the sequence end: zero them so stale or NaN slots cannot reach O
             uint8_t* st = stages + (it % STAGES) * Sh::STAGE_BYTES;
 #pragma unroll
@@ -517,42 +621,43 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&pfull_bar[it & 1]);
-          if (need) named_bar_sync(2, 128);  // the new m_sm is visible before the next tile
+          if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 136 + min((int)it, 31));
 
           if (last) {
-            // ---- segment epilogue: O / l and lse, written to the partial slot ----
+            // ---- segment epilogue: O / l and lse of this warpgroup's heads ----
             const bool oke = mbar_wait(&pvdone_bar[it & 1], (it >> 1) & 1, abort_flag, p.wait_limit_ns);
-            if (named_bar_or(1, 128, !oke || *abort_flag)) { ok = false; ++it; break; }
+            if (named_bar_or(bar_or, 128, !oke || *abort_flag)) { ok = false; ++it; break; }
             tc_fence_after();
-            float lt[NP];
+            float lt[HW];
 #pragma unroll
-            for (int x = 0; x < NP; ++x) lt[x] = l_part[x];
-            warp_reduce_scatter<NP, false>(lt, lane);
-            store_scattered<NP>(lt, red_sm + q4 * NP, lane);
-            named_bar_sync(2, 128);
-            float inv[NP];
+            for (int x = 0; x < HW; ++x) lt[x] = l_part[x];
+            warp_reduce_scatter<HW, false>(lt, lane);
+            store_scattered<HW>(lt, red + q4 * HW, lane);
+            named_bar_sync(bar_sync, 128);
+            float inv[HW];
 #pragma unroll
-            for (int x = 0; x < NP; ++x) {
-              const float l = red_sm[x] + red_sm[NP + x] + red_sm[2 * NP + x] + red_sm[3 * NP + x];
+            for (int x = 0; x < HW; ++x) {
+              const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
               inv[x] = 1.f / l;
-              if (sw == 0 && x % 32 == lane && x < nheads)
-                p.lse_part[(size_t)slot * p.h + head0 + x] = m[x] + __log2f(l);
+              if (sw == 0 && x % 32 == lane && hcol + x < nheads)
+                p.lse_part[(size_t)slot * p.h + head0 + hcol + x] = m[x] + __log2f(l);
             }
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
-              float o[NP];
-              tmem_load_row<NP>(tbase + lane_base + Sh::O_COL + mt * NP, o);
+              float o[HW];
+              tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * NP + hcol, o);
               tmem_ld_wait();
               const int f = mt * 128 + row;
               if (f < Sh::DB) {
-                float* dst = p.o_part + ((size_t)slot * p.h + head0) * Sh::DB + f;
+                float* dst = p.o_part + ((size_t)slot * p.h + head0 + hcol) * Sh::DB + f;
 #pragma unroll
-                for (int x = 0; x < NP; ++x)
-                  if (x < nheads) dst[(size_t)x * Sh::DB] = o[x] * inv[x];
+                for (int x = 0; x < HW; ++x)
+                  if (hcol + x < nheads) dst[(size_t)x * Sh::DB] = o[x] * inv[x];
               }
             }
             tc_fence_before();
-            named_bar_sync(2, 128);  // red_sm and O reads are done before the next segment
+            named_bar_sync(bar_sync, 128);  // red and O reads are done before the next segment
+            if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 168 + min(si, 15));
           }
         }
       }
@@ -561,6 +666,7 @@ __global__ void __launch_bounds__(192, 1)
     if (*abort_flag) break;
   }
 
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 200);
   // ---- teardown: nothing may be in flight when shared memory and TMEM are released ----
   if (warp == 0 && lane == 0) {
     // wait for every stage's last issued load (completed loads return at once)
@@ -580,6 +686,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
   grid_launch_dependents();
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 201);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM_COLS);

@@ -98,22 +98,27 @@ struct mlra_ctx {
 namespace {
 
 // ----- per-variant launch helpers -----
+// Every kernel asks for the largest shared-memory carve-out, so consecutive kernels of a step
+// never make an SM switch its L1 / shared-memory split between them.
+template <class K>
+cudaError_t prep_kernel(K kernel, int smem) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
+}
 template <class Dec>
 cudaError_t prep_decode() {
-  return cudaFuncSetAttribute(mlra_decode_kernel<Dec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Dec::SMEM_BYTES);
+  return prep_kernel(mlra_decode_kernel<Dec>, Dec::SMEM_BYTES);
 }
 template <int DB, int DH, int NT>
 cudaError_t prep_proj() {
   using S = ProjShape<DB, DH, NT>;
-  cudaError_t e = cudaFuncSetAttribute(mlra_absorb_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       S::SMEM1);
+  cudaError_t e = prep_kernel(mlra_absorb_kernel<S>, S::SMEM1);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(mlra_uproj_kernel<S, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           S::SMEM4);
+  e = prep_kernel(mlra_uproj_kernel<S, false>, S::SMEM4);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(mlra_uproj_kernel<S, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              S::SMEM4);
+  return prep_kernel(mlra_uproj_kernel<S, true>, S::SMEM4);
 }
 template <int DB, int DH>
 cudaError_t prep_proj_all() {
@@ -183,7 +188,7 @@ cudaError_t launch_decode(const mlra_ctx* h, const CUtensorMap& mc, const CUtens
                           const CUtensorMap& mqc, const CUtensorMap& mqr, const DecodeParams& dp,
                           cudaStream_t s) {
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->groups * h->nsub), dim3(192), Dec::SMEM_BYTES, s, true, &attr);
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->groups * h->nsub), dim3(Dec::THREADS), Dec::SMEM_BYTES, s, true, &attr);
   return cudaLaunchKernelEx(&c, mlra_decode_kernel<Dec>, mc, mr, mqc, mqr, dp);
 }
 
@@ -518,5 +523,15 @@ int mlra_test_decode_stalled(mlra_handle h, const void* q, mlra_dtype q_dtype, c
   return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, MLRA_F32,
                     nullptr, nullptr, workspace, ws_bytes, stream, 1, wait_limit_ns);
 }
+
+#ifdef MLRA_TRACE
+// Profiling builds only: points the kernels' trace points at a device buffer of
+// [3 kernels][1024 CTAs][256 points] uint64 (NULL turns tracing off).
+int mlra_trace_set(void* device_buffer) {
+  return cudaMemcpyToSymbol(g_mlra_trace, &device_buffer, sizeof(device_buffer)) == cudaSuccess
+             ? MLRA_OK
+             : MLRA_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

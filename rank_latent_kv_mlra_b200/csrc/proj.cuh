@@ -63,7 +63,10 @@ struct ProjShape {
   static constexpr int B1_REG = round_up(NT * AROWB, 1024);
   static constexpr int A1_BOXR = NMT * 128 < 256 ? NMT * 128 : 256;
   static constexpr int A1_TX = NKR * NMT * 128 * AROWB;
-  static constexpr int SMEM1 = NKR * A1_REG + NKR * B1_REG + 1024 + 256;
+  // operand tiles, reused afterwards to stage the output rows
+  static constexpr int STG1 = round_up(NKR * A1_REG + NKR * B1_REG > NT * DB * 2 ? NKR * A1_REG + NKR * B1_REG
+                                                                                  : NT * DB * 2, 1024);
+  static constexpr int SMEM1 = STG1 + 1024 + 256;
   static constexpr int TMEM1 = NMT * NT <= 32 ? 32 : NMT * NT <= 64 ? 64 : NMT * NT <= 128 ? 128 :
                                NMT * NT <= 256 ? 256 : 512;
   // uproj: A = (W^UV_h)^T, MN-major: atoms of AW output columns, each DB rows (K) deep
@@ -76,9 +79,12 @@ struct ProjShape {
   static constexpr int NKB = DB / BW;
   static constexpr int BROWB = BW * 2;
   static constexpr int B4_REG = round_up(NT * BROWB, 1024);
-  static constexpr int SMEM4 = NATOM * ATOM + NKB * B4_REG + 1024 + 1024;
+  static constexpr int STG4 = round_up(NATOM * ATOM + NKB * B4_REG > NT * DH * 4 ? NATOM * ATOM + NKB * B4_REG
+                                                                                  : NT * DH * 4, 1024);
+  static constexpr int SMEM4 = STG4 + 1024 + 1024 + NT * 11 * 4;
   static constexpr int TMEM4 = NT <= 32 ? 32 : NT <= 64 ? 64 : 128;
   static_assert(DH <= 128, "one M tile of head dim");
+
 };
 
 // ---------------------------------------------------------------------------------------
@@ -93,7 +99,7 @@ __global__ void __launch_bounds__(128, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* A = smem;
   uint8_t* Bq = smem + Sh::NKR * Sh::A1_REG;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Bq + Sh::NKR * Sh::B1_REG);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::STG1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -106,6 +112,7 @@ __global__ void __launch_bounds__(128, 1)
   const int sub = blk * p.chunks + hb / p.np;
   const int prow = hb % p.np;
 
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 0);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.status) *p.status = 0;
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
@@ -121,6 +128,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 1);
 
   if (threadIdx.x == 0) {
     tma_prefetch_map(&map_wuk);
@@ -132,49 +140,97 @@ __global__ void __launch_bounds__(128, 1)
                     head * DB + r0, pol);
   }
 
-  // q^C_h for the batch tile -> bf16, K-major swizzled; q^R_h -> packed query (scaled)
-  for (int idx = threadIdx.x; idx < NT * (DH / 8); idx += 128) {
-    const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
-    const int b = n0 + bl;
-    float v[8];
-    if (b < p.batch) {
-      const size_t base = ((size_t)b * p.h + head) * (DH + p.d_r) + d8;
-      if (p.q_f32) {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + base);
-        const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
-        v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-        v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-      } else {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + base));
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  // q^C_h for the batch tile -> bf16, K-major swizzled; q^R_h -> packed query (scaled).
+  // All global loads of a round are issued before any store, so their latencies overlap.
+  {
+    constexpr int QCH = NT * (DH / 8);           // 8-element chunks of q^C
+    constexpr int RND = 8;                        // chunks in flight per thread
+    for (int base = 0; base < QCH; base += 128 * RND) {
+      float v[RND][8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(h2[e]);
-          v[2 * e] = f.x;
-          v[2 * e + 1] = f.y;
+      for (int i = 0; i < RND; ++i) {
+        const int idx = base + i * 128 + threadIdx.x;
+        const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
+        const int b = n0 + bl;
+        if (idx < QCH && b < p.batch) {
+          const size_t off = ((size_t)b * p.h + head) * (DH + p.d_r) + d8;
+          if (p.q_f32) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + off);
+            const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+            v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
+            v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
+          } else {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + off));
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              v[i][2 * e] = f.x;
+              v[i][2 * e + 1] = f.y;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
         }
       }
-    } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      for (int i = 0; i < RND; ++i) {
+        const int idx = base + i * 128 + threadIdx.x;
+        if (idx >= QCH) continue;
+        const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
+        uint4 w;
+        w.x = pack_bf16x2(v[i][0], v[i][1]);
+        w.y = pack_bf16x2(v[i][2], v[i][3]);
+        w.z = pack_bf16x2(v[i][4], v[i][5]);
+        w.w = pack_bf16x2(v[i][6], v[i][7]);
+        *reinterpret_cast<uint4*>(Bq + (d8 / Sh::AW) * Sh::B1_REG +
+                                  swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
+      }
     }
-    uint4 w;
-    w.x = pack_bf16x2(v[0], v[1]);
-    w.y = pack_bf16x2(v[2], v[3]);
-    w.z = pack_bf16x2(v[4], v[5]);
-    w.w = pack_bf16x2(v[6], v[7]);
-    const int kr = d8 / Sh::AW;
-    *reinterpret_cast<uint4*>(Bq + kr * Sh::B1_REG +
-                              swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
-  }
-  for (int idx = threadIdx.x; idx < NT * p.d_r; idx += 128) {
-    const int bl = idx / p.d_r, r = idx % p.d_r;
-    const int b = n0 + bl;
-    if (b >= p.batch) continue;
-    const size_t src = ((size_t)b * p.h + head) * (DH + p.d_r) + DH + r;
-    const float x = p.q_f32 ? __ldg(static_cast<const float*>(p.q) + src)
-                            : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p.q) + src));
-    p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow) * qw + DB + r] = __float2bfloat16_rn(x * p.qscale);
+    // q^R: 8-element chunks, scaled, straight into the packed query
+    const int rch = p.d_r / 8;
+    for (int base = 0; base < NT * rch; base += 128 * 4) {
+      float v[4][8];
+      bool use[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int idx = base + i * 128 + threadIdx.x;
+        const int bl = idx / rch, r8 = (idx % rch) * 8;
+        const int b = n0 + bl;
+        use[i] = idx < NT * rch && b < p.batch;
+        if (use[i]) {
+          const size_t off = ((size_t)b * p.h + head) * (DH + p.d_r) + DH + r8;
+          if (p.q_f32) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + off);
+            const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+            v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
+            v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
+          } else {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + off));
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              v[i][2 * e] = f.x;
+              v[i][2 * e + 1] = f.y;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!use[i]) continue;
+        const int idx = base + i * 128 + threadIdx.x;
+        const int bl = idx / rch, r8 = (idx % rch) * 8;
+        uint4 w;
+        w.x = pack_bf16x2(v[i][0] * p.qscale, v[i][1] * p.qscale);
+        w.y = pack_bf16x2(v[i][2] * p.qscale, v[i][3] * p.qscale);
+        w.z = pack_bf16x2(v[i][4] * p.qscale, v[i][5] * p.qscale);
+        w.w = pack_bf16x2(v[i][6] * p.qscale, v[i][7] * p.qscale);
+        *reinterpret_cast<uint4*>(p.q_pack + (((size_t)(n0 + bl) * p.nsub + sub) * p.np + prow) * qw + DB + r8) = w;
+      }
+    }
   }
   // rows of a head chunk that no head fills (h/k below the MMA width) are zero
   if (hb == p.heads_block - 1 && prow == hb % p.np) {
@@ -189,12 +245,14 @@ __global__ void __launch_bounds__(128, 1)
   }
   fence_proxy_async_smem();
   __syncthreads();
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 2);
 
   if (warp == 0) {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns));
     if (ok) {
       tc_fence_after();
       if (lane == 0) {
+        MLRA_TRACE_POINT(0, 3);
         constexpr uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
         constexpr int KPR = Sh::AW / 16;  // MMA K steps per region
 #pragma unroll
@@ -214,9 +272,13 @@ __global__ void __launch_bounds__(128, 1)
     }
   }
   const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 4);
   if (ok) {
+    // D^T (lanes = latent features, columns = batch rows) -> bf16 rows [b][c] in shared
+    // memory (the weight tile is no longer read), then 16-byte stores of whole rows.
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    __nv_bfloat16* stage_out = reinterpret_cast<__nv_bfloat16*>(A);
 #pragma unroll
     for (int mt = 0; mt < Sh::NMT; ++mt) {
       const int c = mt * 128 + warp * 32 + lane;
@@ -225,16 +287,22 @@ __global__ void __launch_bounds__(128, 1)
       tmem_ld_wait();
       if (c < DB) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          const int b = n0 + n;
-          if (b < p.batch)
-            p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow) * qw + c] =
-                __float2bfloat16_rn(v[n] * p.qscale);
-        }
+        for (int n = 0; n < NT; ++n) stage_out[n * DB + c] = __float2bfloat16_rn(v[n] * p.qscale);
       }
     }
   }
+  __syncthreads();
+  if (ok) {
+    for (int idx = threadIdx.x; idx < NT * (DB / 8); idx += 128) {
+      const int n = idx / (DB / 8), c8 = (idx % (DB / 8)) * 8;
+      const int b = n0 + n;
+      if (b < p.batch)
+        *reinterpret_cast<uint4*>(p.q_pack + (((size_t)b * p.nsub + sub) * p.np + prow) * qw + c8) =
+            *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(A) + n * DB + c8);
+    }
+  }
   // drain before releasing TMEM and shared memory
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 5);
   if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
   tc_fence_before();
   __syncthreads();
@@ -258,7 +326,7 @@ __global__ void __launch_bounds__(128, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* A = smem;
   uint8_t* Bo = smem + Sh::NATOM * Sh::ATOM;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Bo + Sh::NKB * Sh::B4_REG);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::STG4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* err_flag = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));
@@ -269,6 +337,7 @@ __global__ void __launch_bounds__(128, 1)
   const int n0 = blockIdx.y * NT;
   const int warp = warp_id(), lane = lane_id();
   const int cap_len = p.pt_stride * kPage;
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 0);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
@@ -314,54 +383,133 @@ __global__ void __launch_bounds__(128, 1)
   }
   if (err) atomicOr(err_flag, 1);
   __syncthreads();
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 1);
 
   grid_dependency_wait();  // the partials come from the decode kernel
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 2);
 
-  // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major)
-  constexpr int PER = DB / 32;  // features per lane
-  for (int bl = warp; bl < NT; bl += 4) {
+  // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major).
+  // Phase 1: one thread per batch row reads its segments' lse values (all rows at once) and
+  // leaves the merge weights in shared memory. Phase 2: each warp takes rows in rounds and
+  // issues every partial-vector load of a round before the multiply-adds.
+  constexpr int MAXW = 8;  // weights kept per row; longer rows re-read lse in phase 2
+  float* wts = reinterpret_cast<float*>(pref + NT);  // [NT][MAXW]
+  int* rinfo = reinterpret_cast<int*>(wts + NT * MAXW);  // [NT][2]: first slot, count
+  for (int bl = threadIdx.x; bl < NT; bl += blockDim.x) {
     const int b = n0 + bl;
-    float acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    int c0 = 0, nsg = 0;
     float lse2 = -INFINITY;
     if (b < p.batch) {
-      const int n = clamp_len(__ldg(p.seq_lens + b), cap_len, &err);
-      const int tb = tiles_of(n);
+      const int tb = tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err));
       if (tb > 0) {
         const int pb = pref[bl];
-        const int c0 = pb / quota, c1 = (pb + tb - 1) / quota;
-        float mx = -INFINITY;
-        for (int c = c0; c <= c1; ++c) mx = fmaxf(mx, __ldg(p.lse_part + (size_t)(b + c) * p.h + head));
-        float sum = 0.f;
-        for (int c = c0; c <= c1; ++c) sum += exp2f(__ldg(p.lse_part + (size_t)(b + c) * p.h + head) - mx);
-        lse2 = mx + log2f(sum);
-        for (int c = c0; c <= c1; ++c) {
-          const float w = exp2f(__ldg(p.lse_part + (size_t)(b + c) * p.h + head) - lse2);
-          const float* src = p.o_part + ((size_t)(b + c) * p.h + head) * DB + lane * PER;
+        c0 = pb / quota;
+        nsg = (pb + tb - 1) / quota - c0 + 1;
+        float lv[MAXW];
 #pragma unroll
-          for (int e = 0; e < PER; ++e) acc[e] += w * __ldg(src + e);
+        for (int i = 0; i < MAXW; ++i)
+          lv[i] = i < nsg ? __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head) : -INFINITY;
+        float mx = -INFINITY;
+        for (int i = 0; i < nsg; ++i)
+          mx = fmaxf(mx, i < MAXW ? lv[i] : __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head));
+        float sum = 0.f;
+        for (int i = 0; i < nsg; ++i)
+          sum += exp2f((i < MAXW ? lv[i] : __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head)) - mx);
+        lse2 = mx + log2f(sum);
+#pragma unroll
+        for (int i = 0; i < MAXW; ++i) wts[bl * MAXW + i] = i < nsg ? exp2f(lv[i] - lse2) : 0.f;
+      }
+      if (p.lse_out) p.lse_out[(size_t)b * p.h + head] = nsg > 0 ? lse2 * kLn2 : -INFINITY;
+    }
+    rinfo[2 * bl] = c0;
+    rinfo[2 * bl + 1] = nsg;
+    if (nsg > MAXW) wts[bl * MAXW] = lse2;  // long rows: phase 2 recomputes weights from lse
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 3);
+
+  constexpr int PER = DB / 32;  // features per lane
+  constexpr int RB = 4;         // rows per warp per round
+  constexpr int SB = 4;         // segments per row loaded together
+  for (int r0 = warp * RB; r0 < NT; r0 += 4 * RB) {
+    float acc[RB][PER];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[rb][e] = 0.f;
+    int maxseg = 0;
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) maxseg = max(maxseg, r0 + rb < NT ? rinfo[2 * (r0 + rb) + 1] : 0);
+    for (int s0 = 0; s0 < maxseg; s0 += SB) {
+      float v[RB][SB][PER];
+#pragma unroll
+      for (int rb = 0; rb < RB; ++rb) {
+        const int bl = r0 + rb;
+        const int nsg = bl < NT ? rinfo[2 * bl + 1] : 0;
+        const int c0 = bl < NT ? rinfo[2 * bl] : 0;
+#pragma unroll
+        for (int si = 0; si < SB; ++si) {
+          if (s0 + si < nsg) {
+            const float* src = p.o_part + ((size_t)(n0 + bl + c0 + s0 + si) * p.h + head) * DB + lane * PER;
+            if constexpr (PER % 4 == 0) {
+#pragma unroll
+              for (int e = 0; e < PER; e += 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(src + e));
+                v[rb][si][e] = f.x; v[rb][si][e + 1] = f.y; v[rb][si][e + 2] = f.z; v[rb][si][e + 3] = f.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < PER; ++e) v[rb][si][e] = __ldg(src + e);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < PER; ++e) v[rb][si][e] = 0.f;
+          }
         }
       }
-      if (lane == 0 && p.lse_out) p.lse_out[(size_t)b * p.h + head] = tb > 0 ? lse2 * kLn2 : -INFINITY;
-    }
-    if constexpr (LATENT_ONLY) {
-      if (b < p.batch) {
-        float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) dst[e] = acc[e];
+      for (int rb = 0; rb < RB; ++rb) {
+        const int bl = r0 + rb;
+        const int nsg = bl < NT ? rinfo[2 * bl + 1] : 0;
+#pragma unroll
+        for (int si = 0; si < SB; ++si) {
+          const int sidx = s0 + si;
+          if (sidx >= nsg) continue;
+          float wgt;
+          if (nsg <= MAXW) {
+            wgt = wts[bl * MAXW + sidx];
+          } else {
+            const int b = n0 + bl;
+            wgt = exp2f(__ldg(p.lse_part + (size_t)(b + rinfo[2 * bl] + sidx) * p.h + head) - wts[bl * MAXW]);
+          }
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[rb][e] += wgt * v[rb][si][e];
+        }
       }
-    } else {
-      // lane's PER features start at byte lane*PER*2 of the row; write in 2/4/8/16-byte pieces
+    }
 #pragma unroll
-      for (int e = 0; e < PER; e += 2) {
-        const int f = lane * PER + e;
-        uint8_t* reg = Bo + (f / Sh::BW) * Sh::B4_REG;
-        const uint32_t off = swizzle(bl * Sh::BROWB + (f % Sh::BW) * 2, Sh::BROWB);
-        if constexpr (PER == 1) {
-          *reinterpret_cast<__nv_bfloat16*>(reg + off) = __float2bfloat16_rn(acc[0]);
-        } else {
-          *reinterpret_cast<uint32_t*>(reg + off) = pack_bf16x2(acc[e], acc[e + 1]);
+    for (int rb = 0; rb < RB; ++rb) {
+      const int bl = r0 + rb;
+      if (bl >= NT) continue;
+      const int b = n0 + bl;
+      if constexpr (LATENT_ONLY) {
+        if (b < p.batch) {
+          float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) dst[e] = acc[rb][e];
+        }
+      } else {
+        // lane's PER features start at byte lane*PER*2 of the row
+#pragma unroll
+        for (int e = 0; e < PER; e += 2) {
+          const int f = lane * PER + e;
+          uint8_t* reg = Bo + (f / Sh::BW) * Sh::B4_REG;
+          const uint32_t off = swizzle(bl * Sh::BROWB + (f % Sh::BW) * 2, Sh::BROWB);
+          if constexpr (PER == 1) {
+            *reinterpret_cast<__nv_bfloat16*>(reg + off) = __float2bfloat16_rn(acc[rb][0]);
+          } else {
+            *reinterpret_cast<uint32_t*>(reg + off) = pack_bf16x2(acc[rb][e], acc[rb][e + 1]);
+          }
         }
       }
     }
@@ -371,6 +519,7 @@ __global__ void __launch_bounds__(128, 1)
   if constexpr (!LATENT_ONLY) {
     fence_proxy_async_smem();
     __syncthreads();
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 4);
     if (warp == 0) {
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns));
       if (ok) {
@@ -392,25 +541,40 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
     const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 5);
     if (ok) {
+      // D^T (lanes = head-dim d, columns = batch rows) -> rows [b][d] in shared memory (the
+      // operand tiles are no longer read), then 16-byte stores of whole output rows.
       tc_fence_after();
       const int d = warp * 32 + lane;
       float v[NT];
       tmem_load_row<NT>(tbase + (static_cast<uint32_t>(warp * 32) << 16), v);
       tmem_ld_wait();
       if (d < DH) {
+        if (p.out_f32) {
+          float* so = reinterpret_cast<float*>(A);
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          const int b = n0 + n;
-          if (b >= p.batch) continue;
-          const size_t o = ((size_t)b * p.h + head) * DH + d;
-          if (p.out_f32)
-            static_cast<float*>(p.out)[o] = v[n];
-          else
-            static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v[n]);
+          for (int n = 0; n < NT; ++n) so[n * DH + d] = v[n];
+        } else {
+          __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(A);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) so[n * DH + d] = __float2bfloat16_rn(v[n]);
         }
       }
     }
+    __syncthreads();
+    if (ok) {
+      const int esz = p.out_f32 ? 4 : 2;
+      const int chunks = DH * esz / 16;  // 16-byte pieces per output row
+      for (int idx = threadIdx.x; idx < NT * chunks; idx += 128) {
+        const int n = idx / chunks, c = idx % chunks;
+        const int b = n0 + n;
+        if (b < p.batch)
+          *reinterpret_cast<uint4*>(static_cast<char*>(p.out) + (((size_t)b * p.h + head) * DH) * esz + c * 16) =
+              *reinterpret_cast<const uint4*>(A + (size_t)n * DH * esz + c * 16);
+      }
+    }
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 6);
     if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
   }
   tc_fence_before();
