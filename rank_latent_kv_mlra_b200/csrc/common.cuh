@@ -36,7 +36,7 @@ __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 // build); then point `id` of kernel `k` in this CTA records %globaltimer into g_mlra_trace.
 #ifdef MLRA_TRACE
 __device__ unsigned long long* g_mlra_trace;
-constexpr int kTracePoints = 256;
+constexpr int kTracePoints = 512;
 #define MLRA_TRACE_POINT(k, id)                                                              \
   do {                                                                                       \
     const unsigned long long ts_ = global_timer_ns();                                        \
@@ -108,12 +108,15 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
 // Waits until the phase with the given parity of `bar` has completed. Gives up, raising the
 // CTA's abort flag, once `limit_ns` has passed or another role raised the flag. Returns false
 // when it gave up. Every wait in these kernels goes through here, so no wait is endless.
+// The wait polls (test_wait never suspends) with a short sleep between polls: a sleeping
+// warp leaves its issue slots to the warps sharing its scheduler, and wakes within ~0.1 us.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
-  if (mbar_test(bar, parity)) return true;
+  if (mbar_poll(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_test(bar, parity)) return true;
+    __nanosleep(32);
+    if (mbar_poll(bar, parity)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -127,7 +130,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_test(bar, parity)) {
+  while (!mbar_poll(bar, parity)) {
+    __nanosleep(32);
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
   return true;
@@ -512,6 +516,80 @@ __device__ __forceinline__ int block_collect_segments(const int* __restrict__ se
   *resume_b = res_b;
   *resume_p = res_p;
   return count;
+}
+
+// One-pass planning for batches up to blockDim.x * kPlanPer sequences: each thread keeps the
+// lengths of its contiguous run of sequences in registers, so seq_lens is read once (one
+// memory round trip) instead of once per pass.
+constexpr int kPlanPer = 8;
+struct PlanRegs {
+  int n[kPlanPer];  // lengths (clamped) of sequences base .. base + per - 1
+  int base, per;
+  int first_p;      // flattened tile index where sequence `base` starts
+  int total;        // T = sum of tiles over all sequences
+};
+
+// All threads call it. Returns false (and loads nothing) when the batch is too large for
+// the register plan; callers then use the multi-pass routines above.
+__device__ __forceinline__ bool block_plan_load(const int* __restrict__ seq_lens, int batch, int cap_len,
+                                                PlanRegs& pr, int* scratch, int* err) {
+  pr.per = (batch + blockDim.x - 1) / blockDim.x;
+  if (pr.per > kPlanPer) return false;
+  pr.base = threadIdx.x * pr.per;
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < kPlanPer; ++i) {
+    const int b = pr.base + i;
+    pr.n[i] = (i < pr.per && b < batch) ? clamp_len(__ldg(seq_lens + b), cap_len, err) : 0;
+    local += tiles_of(pr.n[i]);
+  }
+  pr.first_p = block_scan_tiles(local, scratch, &pr.total);
+  return true;
+}
+
+// Segments of the flattened tile range [lo, hi) from a register plan; same result and order
+// as block_collect_segments. Writes at most cap_list entries; returns the number of segments
+// in the range (which may exceed cap_list: then the caller resumes with the multi-pass
+// routine from (*resume_b, *resume_p)).
+__device__ __forceinline__ int block_plan_segments(const PlanRegs& pr, int lo, int hi, Segment* list, int cap_list,
+                                                   int* scratch, int* resume_b, int* resume_p) {
+  int hits = 0;
+  int pb = pr.first_p;
+#pragma unroll
+  for (int i = 0; i < kPlanPer; ++i) {
+    const int t = tiles_of(pr.n[i]);
+    if (i < pr.per && t > 0 && pb < hi && pb + t > lo) ++hits;
+    pb += t;
+  }
+  int total_hits;
+  int ord = block_scan_tiles(hits, scratch, &total_hits);
+  pb = pr.first_p;
+#pragma unroll
+  for (int i = 0; i < kPlanPer; ++i) {
+    const int t = tiles_of(pr.n[i]);
+    if (i < pr.per && t > 0 && pb < hi && pb + t > lo) {
+      if (ord < cap_list) {
+        Segment sg;
+        sg.b = pr.base + i;
+        sg.tile_begin = max(lo, pb) - pb;
+        sg.tile_end = min(hi, pb + t) - pb;
+        sg.n = pr.n[i];
+        list[ord] = sg;
+      } else if (ord == cap_list) {
+        scratch[34] = pr.base + i;
+        scratch[35] = pb;
+      }
+      ++ord;
+    }
+    pb += t;
+  }
+  __syncthreads();
+  if (total_hits > cap_list) {
+    *resume_b = scratch[34];
+    *resume_p = scratch[35];
+  }
+  __syncthreads();
+  return total_hits;
 }
 
 }  // namespace mlra

@@ -252,11 +252,16 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 1);
+  // the combine kernel may be scheduled as soon as SMs free up; it waits for this grid's
+  // partials before reading them
+  grid_launch_dependents();
 
   // ---- plan: which flattened tiles this group owns (seq_lens do not depend on the
   // previous kernel, so this overlaps its tail under programmatic dependent launch) ----
   int err = 0;
-  const int T = block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
+  PlanRegs pr;
+  const bool reg_plan = block_plan_load(p.seq_lens, p.batch, cap_len, pr, scratch, &err);
+  const int T = reg_plan ? pr.total : block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
   const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
   const int lo = min(group * quota, T);
   const int hi = min(lo + quota, T);
@@ -274,11 +279,20 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 
   int b_start = 0, p_start = 0;
   bool more = lo < hi;
+  bool first_list = true;
   while (more) {
-    int more_i, rb, rp;
-    const int nseg = block_collect_segments(p.seq_lens, p.batch, cap_len, lo, hi, b_start, p_start,
-                                            segs, Sh::MAX_SEGS, scratch, &more_i, &rb, &rp, &err);
-    more = more_i != 0;
+    int nseg, rb = p.batch, rp = 0;
+    if (first_list && reg_plan) {
+      const int total = block_plan_segments(pr, lo, hi, segs, Sh::MAX_SEGS, scratch, &rb, &rp);
+      nseg = min(total, Sh::MAX_SEGS);
+      more = total > Sh::MAX_SEGS;
+    } else {
+      int more_i;
+      nseg = block_collect_segments(p.seq_lens, p.batch, cap_len, lo, hi, b_start, p_start, segs,
+                                    Sh::MAX_SEGS, scratch, &more_i, &rb, &rp, &err);
+      more = more_i != 0;
+    }
+    first_list = false;
     b_start = rb;
     p_start = rp;
     if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 2);
@@ -472,7 +486,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           if (issued) {
             t_idle = 0;
           } else {
-            // nothing ready: bounded wait, like every other wait in this kernel
+            // nothing ready: sleep briefly (leaves issue slots to the softmax warps on this
+            // scheduler), bounded like every other wait in this kernel
+            __nanosleep(32);
             if (*abort_flag) break;
             const uint64_t now = global_timer_ns();
             if (t_idle == 0) {
@@ -522,6 +538,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             okl = okl && mbar_wait(&pvdone_bar[j & 1], (j >> 1) & 1, abort_flag, p.wait_limit_ns);
           }
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 104 + min((int)it, 31));
+          if (warp == 6 && lane == 0) MLRA_TRACE_POINT(1, 320 + min((int)it, 31));
           tc_fence_after();
           float s[HW];
           tmem_load_row<HW>(tbase + lane_base + Sh::S_COL0 + (it & 1) * NP + hcol, s);
@@ -554,6 +571,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           for (int x = 0; x < HW; ++x) pr[x] = fast_exp2(xs[x]);
 
           const bool need = named_bar_or(bar_or, 128, !okl || first || dm[0] > kRescaleSlack);
+          if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 256 + min((int)it, 31));
           if (need) {
             if (named_bar_or(bar_or, 128, !okl || *abort_flag)) { ok = false; break; }
             float tmax[HW];
@@ -622,6 +640,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&pfull_bar[it & 1]);
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 136 + min((int)it, 31));
+          if (warp == 6 && lane == 0) MLRA_TRACE_POINT(1, 288 + min((int)it, 31));
 
           if (last) {
             // ---- segment epilogue: O / l and lse of this warpgroup's heads ----
@@ -657,7 +676,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             }
             tc_fence_before();
             named_bar_sync(bar_sync, 128);  // red and O reads are done before the next segment
-            if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 168 + min(si, 15));
+            if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 168 + min(si, 7));
           }
         }
       }
@@ -685,7 +704,6 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
-  grid_launch_dependents();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 201);
   if (warp == 1) {
     tc_fence_after();

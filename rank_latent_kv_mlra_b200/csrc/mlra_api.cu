@@ -9,6 +9,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -393,6 +394,12 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
       if (e == cudaSuccess) e = prep_decode<DecMlra4q2>();
       if (e == cudaSuccess) e = prep_proj_all<128, 128>();
       h->stages = DecMlra4::STAGES;
+      {
+        // tuning switch: MLRA_DECODE_STAGES=3 selects the 3-stage pipeline with two query
+        // buffers (no bubble at segment changes) instead of 4 stages with one
+        const char* env = std::getenv("MLRA_DECODE_STAGES");
+        if (env != nullptr && std::atoi(env) == DecMlra4q2::STAGES) h->stages = DecMlra4q2::STAGES;
+      }
       break;
     case kMlra2:
       e = prep_decode<DecMlra2>();
@@ -526,7 +533,29 @@ int mlra_test_decode_stalled(mlra_handle h, const void* q, mlra_dtype q_dtype, c
 
 #ifdef MLRA_TRACE
 // Profiling builds only: points the kernels' trace points at a device buffer of
-// [3 kernels][1024 CTAs][256 points] uint64 (NULL turns tracing off).
+// [3 kernels][1024 CTAs][512 points] uint64 (NULL turns tracing off).
+// Profiling builds only: one launch of the absorb kernel alone (same arguments as a decode).
+int mlra_trace_absorb_only(mlra_handle h, const void* q, int batch, void* workspace, void* stream) {
+  Workspace w = carve(h, batch, workspace);
+  ProjParams pp = {};
+  pp.q = q;
+  pp.q_f32 = 0;
+  pp.q_pack = w.q_pack;
+  pp.qscale = h->scale * kLog2e;
+  pp.d_r = h->d_r;
+  pp.np = h->np;
+  pp.nsub = h->nsub;
+  pp.chunks = h->chunks;
+  pp.heads_block = h->heads_block;
+  pp.batch = batch;
+  pp.h = h->cfg.h;
+  pp.status = w.status;
+  pp.wait_limit_ns = kWaitLimitNs;
+  if (h->var != kMlra4) return MLRA_ERR_UNSUPPORTED;
+  return dispatch_absorb<128, 128>(h, pp, batch, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MLRA_OK
+                                                                                                   : MLRA_ERR_CUDA;
+}
+
 int mlra_trace_set(void* device_buffer) {
   return cudaMemcpyToSymbol(g_mlra_trace, &device_buffer, sizeof(device_buffer)) == cudaSuccess
              ? MLRA_OK

@@ -129,6 +129,9 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 1);
+  // let the decode kernel's CTAs start (on SMs this grid leaves free) and run their set-up and
+  // split planning now; they wait for this grid's results before reading them
+  grid_launch_dependents();
 
   if (threadIdx.x == 0) {
     tma_prefetch_map(&map_wuk);
@@ -140,20 +143,26 @@ __global__ void __launch_bounds__(128, 1)
                     head * DB + r0, pol);
   }
 
-  // q^C_h for the batch tile -> bf16, K-major swizzled; q^R_h -> packed query (scaled).
-  // All global loads of a round are issued before any store, so their latencies overlap.
+  // q_h for the batch tile, in 8-element chunks: q^C chunks -> bf16, K-major swizzled tile
+  // (the MMA's B operand); q^R chunks -> packed query, scaled. All global loads of a round are
+  // issued before any store, so the round costs one memory round trip.
   {
-    constexpr int QCH = NT * (DH / 8);           // 8-element chunks of q^C
-    constexpr int RND = 8;                        // chunks in flight per thread
-    for (int base = 0; base < QCH; base += 128 * RND) {
+    const int qwh = DH + p.d_r;        // elements of one q row
+    const int cpr = qwh / 8;           // chunks per row
+    const int nch = NT * cpr;
+    constexpr int RND = 8;
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 10);
+    for (int base = 0; base < nch; base += 128 * RND) {
       float v[RND][8];
+      bool use[RND];
 #pragma unroll
       for (int i = 0; i < RND; ++i) {
         const int idx = base + i * 128 + threadIdx.x;
-        const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
+        const int bl = idx / cpr, d8 = (idx % cpr) * 8;
         const int b = n0 + bl;
-        if (idx < QCH && b < p.batch) {
-          const size_t off = ((size_t)b * p.h + head) * (DH + p.d_r) + d8;
+        use[i] = idx < nch;
+        if (use[i] && b < p.batch) {
+          const size_t off = ((size_t)b * p.h + head) * qwh + d8;
           if (p.q_f32) {
             const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + off);
             const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
@@ -176,62 +185,30 @@ __global__ void __launch_bounds__(128, 1)
       }
 #pragma unroll
       for (int i = 0; i < RND; ++i) {
-        const int idx = base + i * 128 + threadIdx.x;
-        if (idx >= QCH) continue;
-        const int bl = idx / (DH / 8), d8 = (idx % (DH / 8)) * 8;
-        uint4 w;
-        w.x = pack_bf16x2(v[i][0], v[i][1]);
-        w.y = pack_bf16x2(v[i][2], v[i][3]);
-        w.z = pack_bf16x2(v[i][4], v[i][5]);
-        w.w = pack_bf16x2(v[i][6], v[i][7]);
-        *reinterpret_cast<uint4*>(Bq + (d8 / Sh::AW) * Sh::B1_REG +
-                                  swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
-      }
-    }
-    // q^R: 8-element chunks, scaled, straight into the packed query
-    const int rch = p.d_r / 8;
-    for (int base = 0; base < NT * rch; base += 128 * 4) {
-      float v[4][8];
-      bool use[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int idx = base + i * 128 + threadIdx.x;
-        const int bl = idx / rch, r8 = (idx % rch) * 8;
-        const int b = n0 + bl;
-        use[i] = idx < NT * rch && b < p.batch;
-        if (use[i]) {
-          const size_t off = ((size_t)b * p.h + head) * (DH + p.d_r) + DH + r8;
-          if (p.q_f32) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + off);
-            const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
-            v[i][0] = x0.x; v[i][1] = x0.y; v[i][2] = x0.z; v[i][3] = x0.w;
-            v[i][4] = x1.x; v[i][5] = x1.y; v[i][6] = x1.z; v[i][7] = x1.w;
-          } else {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + off));
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(h2[e]);
-              v[i][2 * e] = f.x;
-              v[i][2 * e + 1] = f.y;
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
         if (!use[i]) continue;
         const int idx = base + i * 128 + threadIdx.x;
-        const int bl = idx / rch, r8 = (idx % rch) * 8;
-        uint4 w;
-        w.x = pack_bf16x2(v[i][0] * p.qscale, v[i][1] * p.qscale);
-        w.y = pack_bf16x2(v[i][2] * p.qscale, v[i][3] * p.qscale);
-        w.z = pack_bf16x2(v[i][4] * p.qscale, v[i][5] * p.qscale);
-        w.w = pack_bf16x2(v[i][6] * p.qscale, v[i][7] * p.qscale);
-        *reinterpret_cast<uint4*>(p.q_pack + (((size_t)(n0 + bl) * p.nsub + sub) * p.np + prow) * qw + DB + r8) = w;
+        const int bl = idx / cpr, d8 = (idx % cpr) * 8;
+        if (d8 < DH) {
+          uint4 w;
+          w.x = pack_bf16x2(v[i][0], v[i][1]);
+          w.y = pack_bf16x2(v[i][2], v[i][3]);
+          w.z = pack_bf16x2(v[i][4], v[i][5]);
+          w.w = pack_bf16x2(v[i][6], v[i][7]);
+          *reinterpret_cast<uint4*>(Bq + (d8 / Sh::AW) * Sh::B1_REG +
+                                    swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
+        } else if (n0 + bl < p.batch) {
+          uint4 w;
+          w.x = pack_bf16x2(v[i][0] * p.qscale, v[i][1] * p.qscale);
+          w.y = pack_bf16x2(v[i][2] * p.qscale, v[i][3] * p.qscale);
+          w.z = pack_bf16x2(v[i][4] * p.qscale, v[i][5] * p.qscale);
+          w.w = pack_bf16x2(v[i][6] * p.qscale, v[i][7] * p.qscale);
+          *reinterpret_cast<uint4*>(p.q_pack + (((size_t)(n0 + bl) * p.nsub + sub) * p.np + prow) * qw + DB +
+                                    (d8 - DH)) = w;
+        }
       }
     }
   }
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 11);
   // rows of a head chunk that no head fills (h/k below the MMA width) are zero
   if (hb == p.heads_block - 1 && prow == hb % p.np) {
     const int pad = p.np - 1 - prow;
@@ -243,7 +220,9 @@ __global__ void __launch_bounds__(128, 1)
           __float2bfloat16_rn(0.f);
     }
   }
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 12);
   fence_proxy_async_smem();
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 13);
   __syncthreads();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 2);
 
@@ -307,7 +286,6 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
-  grid_launch_dependents();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM1);
@@ -368,9 +346,19 @@ __global__ void __launch_bounds__(128, 1)
 
   // plan: total tiles and the flattened start of each sequence of this batch tile
   int err = 0;
-  const int T = block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
-  const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
-  {
+  PlanRegs pr;
+  int T;
+  if (block_plan_load(p.seq_lens, p.batch, cap_len, pr, scratch, &err)) {
+    T = pr.total;
+    int pb = pr.first_p;
+#pragma unroll
+    for (int i = 0; i < kPlanPer; ++i) {
+      const int b = pr.base + i;
+      if (i < pr.per && b >= n0 && b < n0 + NT) pref[b - n0] = pb;
+      pb += tiles_of(pr.n[i]);
+    }
+  } else {
+    T = block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
     int running = 0;
     for (int base = 0; base < min(p.batch, n0 + NT); base += blockDim.x) {
       const int b = base + threadIdx.x;
@@ -381,6 +369,7 @@ __global__ void __launch_bounds__(128, 1)
       running += chunk_total;
     }
   }
+  const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
   if (err) atomicOr(err_flag, 1);
   __syncthreads();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 1);
@@ -389,68 +378,52 @@ __global__ void __launch_bounds__(128, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 2);
 
   // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major).
-  // Phase 1: one thread per batch row reads its segments' lse values (all rows at once) and
-  // leaves the merge weights in shared memory. Phase 2: each warp takes rows in rounds and
-  // issues every partial-vector load of a round before the multiply-adds.
-  constexpr int MAXW = 8;  // weights kept per row; longer rows re-read lse in phase 2
-  float* wts = reinterpret_cast<float*>(pref + NT);  // [NT][MAXW]
-  int* rinfo = reinterpret_cast<int*>(wts + NT * MAXW);  // [NT][2]: first slot, count
-  for (int bl = threadIdx.x; bl < NT; bl += blockDim.x) {
-    const int b = n0 + bl;
-    int c0 = 0, nsg = 0;
-    float lse2 = -INFINITY;
-    if (b < p.batch) {
-      const int tb = tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err));
-      if (tb > 0) {
-        const int pb = pref[bl];
-        c0 = pb / quota;
-        nsg = (pb + tb - 1) / quota - c0 + 1;
-        float lv[MAXW];
-#pragma unroll
-        for (int i = 0; i < MAXW; ++i)
-          lv[i] = i < nsg ? __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head) : -INFINITY;
-        float mx = -INFINITY;
-        for (int i = 0; i < nsg; ++i)
-          mx = fmaxf(mx, i < MAXW ? lv[i] : __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head));
-        float sum = 0.f;
-        for (int i = 0; i < nsg; ++i)
-          sum += exp2f((i < MAXW ? lv[i] : __ldg(p.lse_part + (size_t)(b + c0 + i) * p.h + head)) - mx);
-        lse2 = mx + log2f(sum);
-#pragma unroll
-        for (int i = 0; i < MAXW; ++i) wts[bl * MAXW + i] = i < nsg ? exp2f(lv[i] - lse2) : 0.f;
-      }
-      if (p.lse_out) p.lse_out[(size_t)b * p.h + head] = nsg > 0 ? lse2 * kLn2 : -INFINITY;
-    }
-    rinfo[2 * bl] = c0;
-    rinfo[2 * bl + 1] = nsg;
-    if (nsg > MAXW) wts[bl * MAXW] = lse2;  // long rows: phase 2 recomputes weights from lse
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 3);
-
+  // Each warp takes RB batch rows at a time and issues every load of a round (the rows'
+  // lse values and partial vectors, up to SB segments each) before using any of them, so a
+  // round costs one memory round trip. Rows with more segments take further rounds.
   constexpr int PER = DB / 32;  // features per lane
   constexpr int RB = 4;         // rows per warp per round
   constexpr int SB = 4;         // segments per row loaded together
   for (int r0 = warp * RB; r0 < NT; r0 += 4 * RB) {
-    float acc[RB][PER];
+    int c0[RB], nsg[RB];
 #pragma unroll
-    for (int rb = 0; rb < RB; ++rb)
+    for (int rb = 0; rb < RB; ++rb) {
+      const int bl = r0 + rb, b = n0 + bl;
+      c0[rb] = 0;
+      nsg[rb] = 0;
+      if (bl < NT && b < p.batch) {
+        const int tb = tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err));
+        if (tb > 0) {
+          const int pb = pref[bl];
+          c0[rb] = pb / quota;
+          nsg[rb] = (pb + tb - 1) / quota - c0[rb] + 1;
+        }
+      }
+    }
+    float acc[RB][PER];
+    float mx[RB], sum[RB];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+      mx[rb] = -INFINITY;
+      sum[rb] = 0.f;
 #pragma unroll
       for (int e = 0; e < PER; ++e) acc[rb][e] = 0.f;
+    }
     int maxseg = 0;
 #pragma unroll
-    for (int rb = 0; rb < RB; ++rb) maxseg = max(maxseg, r0 + rb < NT ? rinfo[2 * (r0 + rb) + 1] : 0);
+    for (int rb = 0; rb < RB; ++rb) maxseg = max(maxseg, nsg[rb]);
     for (int s0 = 0; s0 < maxseg; s0 += SB) {
+      float lv[RB][SB];
       float v[RB][SB][PER];
 #pragma unroll
       for (int rb = 0; rb < RB; ++rb) {
-        const int bl = r0 + rb;
-        const int nsg = bl < NT ? rinfo[2 * bl + 1] : 0;
-        const int c0 = bl < NT ? rinfo[2 * bl] : 0;
+        const int b = n0 + r0 + rb;
 #pragma unroll
         for (int si = 0; si < SB; ++si) {
-          if (s0 + si < nsg) {
-            const float* src = p.o_part + ((size_t)(n0 + bl + c0 + s0 + si) * p.h + head) * DB + lane * PER;
+          if (s0 + si < nsg[rb]) {
+            const size_t slot = (size_t)(b + c0[rb] + s0 + si);
+            lv[rb][si] = __ldg(p.lse_part + slot * p.h + head);
+            const float* src = p.o_part + (slot * p.h + head) * DB + lane * PER;
             if constexpr (PER % 4 == 0) {
 #pragma unroll
               for (int e = 0; e < PER; e += 4) {
@@ -462,36 +435,42 @@ __global__ void __launch_bounds__(128, 1)
               for (int e = 0; e < PER; ++e) v[rb][si][e] = __ldg(src + e);
             }
           } else {
+            lv[rb][si] = -INFINITY;
 #pragma unroll
             for (int e = 0; e < PER; ++e) v[rb][si][e] = 0.f;
           }
         }
       }
+      // online log-sum-exp merge (base 2) of this round's segments
 #pragma unroll
       for (int rb = 0; rb < RB; ++rb) {
-        const int bl = r0 + rb;
-        const int nsg = bl < NT ? rinfo[2 * bl + 1] : 0;
+        float m_new = mx[rb];
+#pragma unroll
+        for (int si = 0; si < SB; ++si) m_new = fmaxf(m_new, lv[rb][si]);
+        if (m_new == -INFINITY) continue;
+        const float sc = exp2f(mx[rb] - m_new);  // 0 when mx was -inf
+        sum[rb] *= sc;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[rb][e] *= sc;
 #pragma unroll
         for (int si = 0; si < SB; ++si) {
-          const int sidx = s0 + si;
-          if (sidx >= nsg) continue;
-          float wgt;
-          if (nsg <= MAXW) {
-            wgt = wts[bl * MAXW + sidx];
-          } else {
-            const int b = n0 + bl;
-            wgt = exp2f(__ldg(p.lse_part + (size_t)(b + rinfo[2 * bl] + sidx) * p.h + head) - wts[bl * MAXW]);
-          }
+          const float wgt = exp2f(lv[rb][si] - m_new);  // 0 for absent segments
+          sum[rb] += wgt;
 #pragma unroll
           for (int e = 0; e < PER; ++e) acc[rb][e] += wgt * v[rb][si][e];
         }
+        mx[rb] = m_new;
       }
     }
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
-      const int bl = r0 + rb;
+      const int bl = r0 + rb, b = n0 + bl;
       if (bl >= NT) continue;
-      const int b = n0 + bl;
+      const float inv = sum[rb] > 0.f ? 1.f / sum[rb] : 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[rb][e] *= inv;
+      if (b < p.batch && lane == 0 && p.lse_out)
+        p.lse_out[(size_t)b * p.h + head] = nsg[rb] > 0 ? (mx[rb] + log2f(sum[rb])) * kLn2 : -INFINITY;
       if constexpr (LATENT_ONLY) {
         if (b < p.batch) {
           float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
@@ -514,6 +493,7 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
+  if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 3);
   if (err) atomicOr(err_flag, 1);
 
   if constexpr (!LATENT_ONLY) {
