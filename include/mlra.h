@@ -18,8 +18,9 @@
  * Conventions shared by every entry point:
  *   - Device pointers are CUDA global memory on the current device; host pointers are marked.
  *   - The caller owns every buffer. The library allocates no device memory: scratch lives in
- *     the caller's workspace (mlra_workspace_size). A handle borrows the weight pointers
- *     until mlra_destroy.
+ *     the caller's workspace (mlra_workspace_size), except for mlra_decode_noalloc, whose
+ *     scratch is one fixed 16 MiB device array of the library. A handle borrows the weight
+ *     pointers until mlra_destroy.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream). No entry
  *     point synchronises, except mlra_get_status.
  *   - Return values are mlra_status codes. Argument errors are found on the host before any
@@ -48,7 +49,8 @@ typedef enum {
   MLRA_ERR_PAGE_OOB = -4,      /* device: a page-table entry outside [0, num_pages) */
   MLRA_ERR_TIMEOUT = -5,       /* device: a pipeline wait passed its time limit */
   MLRA_ERR_WORKSPACE = -6,     /* workspace smaller than mlra_workspace_size */
-  MLRA_ERR_SEQ_LEN = -7        /* device: seq_len < 0 or > pt_stride * page_size */
+  MLRA_ERR_SEQ_LEN = -7,       /* device: seq_len < 0 or > pt_stride * page_size */
+  MLRA_ERR_SCRATCH_LIMIT = -8  /* mlra_decode_noalloc: batch too large for its fixed scratch */
 } mlra_status;
 
 typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype;
@@ -100,6 +102,29 @@ int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* po
                 int num_pages, const int32_t* page_table, int pt_stride,
                 const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
                 float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* mlra_decode for callers that cannot allocate device memory when they decode (a serving
+ * engine whose KV-cache pool took all HBM left after the weights, a plug-in inside a runtime
+ * that owns every allocation): no workspace argument, and nothing is allocated. The papers
+ * have no counterpart: this is a property of the library, not of the method.
+ *   Scratch: one 16 MiB device array inside the library (a static __device__ object), held
+ *     by every GPU that loads the library until the process exits. Enough for
+ *     mlra_workspace_size(batch) <= 16 MiB, i.e. MLRA-4 with 128 heads up to batch 124 on 148 SMs;
+ *     larger requests return MLRA_ERR_SCRATCH_LIMIT before any launch.
+ *   First call on a device: looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current and keeps it. Make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's
+ *     contents; each call clears the status word it needs at zero. Calls whose kernels
+ *     overlap on the GPU (other streams, threads or handles) race on the array: serialise
+ *     them.
+ *   status: device int32 word, or NULL. Receives this call's device status (0 = OK, else an
+ *     mlra_status code) once the kernels have finished, in stream order. With NULL, device
+ *     errors of this call are not reported.
+ * All other arguments, layouts and results are those of mlra_decode. */
+int mlra_decode_noalloc(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
+                        int num_pages, const int32_t* page_table, int pt_stride,
+                        const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
+                        float* lse, int32_t* status, void* stream);
 
 /* Same as mlra_decode but stops before the up-projection: latent_out receives the
  * normalised latent output o~ as device fp32 [batch][h][d_c/k], lse as above (nullable).

@@ -29,12 +29,13 @@ STATUS = {
     -5: "MLRA_ERR_TIMEOUT",
     -6: "MLRA_ERR_WORKSPACE",
     -7: "MLRA_ERR_SEQ_LEN",
+    -8: "MLRA_ERR_SCRATCH_LIMIT",
 }
 
 EXPORTED = [
     "mlra_create", "mlra_destroy", "mlra_workspace_size", "mlra_decode", "mlra_decode_latent",
     "mlra_append_cache", "mlra_plan", "mlra_get_info", "mlra_get_status", "mlra_status_string",
-    "mlra_decode_profiled",
+    "mlra_decode_profiled", "mlra_decode_noalloc",
 ]
 
 
@@ -74,6 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mlra_destroy.restype = None
     lib.mlra_workspace_size.argtypes = [P, I, ctypes.POINTER(S)]
     lib.mlra_decode.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, S, P]
+    lib.mlra_decode_noalloc.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, P]
     lib.mlra_decode_latent.argtypes = [P, P, I, P, I, P, I, P, I, P, P, P, S, P]
     lib.mlra_decode_profiled.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, S, P, P]
     lib.mlra_append_cache.argtypes = [P, P, I, P, I, I, P, P, P, P, I, I, P, P]
@@ -194,6 +196,36 @@ def mlra_decode(handle: Handle, q, pool, page_table, seq_lens, out, lse=None, wo
         page_table.shape[1], _ptr(seq_lens), B, _ptr(out), _dtype(out), _ptr(lse), _ptr(workspace),
         workspace.numel(), _stream(stream)), "mlra_decode")
     return workspace
+
+
+def mlra_decode_noalloc(handle: Handle, q, pool, page_table, seq_lens, out, lse=None, status=None,
+                        stream=None):
+    """mlra_decode without a workspace: the scratch is the library's fixed 16 MiB device array,
+    shared by every call on the device, so calls must not overlap on the GPU. For callers that
+    cannot allocate device memory while decoding. `status` is an optional device int32 tensor
+    that receives the call's device status. Raises MlraError(MLRA_ERR_SCRATCH_LIMIT) for a
+    batch the array cannot hold."""
+    _require(q, "q")
+    _require(pool, "pool", torch.bfloat16)
+    _require(page_table, "page_table", torch.int32)
+    _require(seq_lens, "seq_lens", torch.int32)
+    _require(out, "out")
+    if lse is not None:
+        _require(lse, "lse", torch.float32)
+    if status is not None:
+        _require(status, "status", torch.int32)
+    cfg = handle.cfg
+    B = q.shape[0]
+    if tuple(q.shape) != (B, cfg.h, cfg.d_h + cfg.d_rope):
+        raise ValueError("q must be [batch][h][d_h + d_rope]")
+    if pool.dim() != 3 or pool.shape[1] != cfg.page_size or pool.shape[2] != cfg.d_c + cfg.d_rope:
+        raise ValueError("pool must be [num_pages][page_size][d_c + d_rope]")
+    if page_table.dim() != 2 or page_table.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("page_table must be [batch][pt_stride], seq_lens [batch]")
+    _check(load_library().mlra_decode_noalloc(
+        handle.ptr, _ptr(q), _dtype(q), _ptr(pool), pool.shape[0], _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, _ptr(out), _dtype(out), _ptr(lse), _ptr(status),
+        _stream(stream)), "mlra_decode_noalloc")
 
 
 def mlra_decode_profiled(handle: Handle, q, pool, page_table, seq_lens, out, events, lse=None,

@@ -341,6 +341,47 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   return e == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------------------
+// Scratch of mlra_decode_noalloc: mlra_decode with its workspace in a fixed device array of
+// this library instead of one the caller passes. It exists for callers that cannot allocate
+// device memory at the point where they decode: a serving engine that has handed all free
+// HBM to its KV-cache page pool once the weights were loaded (a per-step allocation would
+// fail, or would force the pool to shrink), or a plug-in that runs inside another runtime
+// which owns every allocation and hands it only the tensors of the step.
+//
+// kNoAllocScratchBytes is the whole array; every GPU that loads this library holds it until
+// the process exits. It covers mlra_workspace_size(batch) for MLRA-4 with 128 heads up to
+// batch 124 on a 148-SM GPU. All calls on a device share the one array and it keeps what the
+// last call left there, so each call clears the status word (every other byte the kernels
+// read is written earlier in the same call). Calls whose kernels overlap on the GPU (other
+// streams, other threads, other handles on the same device) race on it.
+// ---------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on `dev`, which must be the current device. In host
+// code the array's name only identifies the symbol; the address is looked up once per device
+// (the first mlra_decode_noalloc call there) and kept.
+int noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MLRA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return MLRA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLRA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -443,6 +484,26 @@ int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* po
                     lse, nullptr, workspace, ws_bytes, stream, 0, kWaitLimitNs);
 }
 
+int mlra_decode_noalloc(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
+                        const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch,
+                        void* out, mlra_dtype out_dtype, float* lse, int32_t* status, void* stream) {
+  if (!h || !out || batch <= 0 || batch > 4096) return MLRA_ERR_INVALID_ARG;
+  if (carve(h, batch, nullptr).bytes > kNoAllocScratchBytes) return MLRA_ERR_SCRATCH_LIMIT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MLRA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(dev, &scratch);
+  if (rc != MLRA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  rc = run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, out_dtype, lse,
+                  nullptr, scratch, kNoAllocScratchBytes, stream, 0, kWaitLimitNs);
+  if (rc != MLRA_OK) return rc;
+  if (status && cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+
 int mlra_decode_latent(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool, int num_pages,
                        const int32_t* page_table, int pt_stride, const int32_t* seq_lens, int batch,
                        float* latent_out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
@@ -504,6 +565,7 @@ const char* mlra_status_string(int code) {
     case MLRA_ERR_TIMEOUT: return "device pipeline wait timed out";
     case MLRA_ERR_WORKSPACE: return "workspace too small";
     case MLRA_ERR_SEQ_LEN: return "sequence length outside its page-table row";
+    case MLRA_ERR_SCRATCH_LIMIT: return "batch needs more than the 16 MiB fixed scratch of mlra_decode_noalloc";
     default: return "unknown status";
   }
 }
