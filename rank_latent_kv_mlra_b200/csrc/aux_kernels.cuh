@@ -50,19 +50,41 @@ __global__ void __launch_bounds__(192, 1)
                      int* __restrict__ out, int max_segments, int* __restrict__ count, int* status) {
   __shared__ Segment list[64];
   __shared__ int scratch[40];
+  __shared__ int words[3];
   int err = 0;
   const int cap_len = pt_stride * kPage;
-  const int T = block_total_tiles(seq_lens, batch, cap_len, scratch, &err);
+  // the decode kernel's planning: warp scan for small batches, block scans otherwise
+  WarpPlan wp;
+  const bool warp_plan = warp_plan_load(seq_lens, batch, cap_len, wp, &err);
+  const int T = warp_plan ? wp.total : block_total_tiles(seq_lens, batch, cap_len, scratch, &err);
   const int quota = T > 0 ? (T + groups - 1) / groups : 1;
   int written = 0;
   for (int g = 0; g < groups; ++g) {
     const int lo = min(g * quota, T), hi = min(lo + quota, T);
     if (lo >= hi) break;
     int b_start = 0, p_start = 0, more = 1;
+    bool first = true;
     while (more) {
-      int rb, rp;
-      const int n = block_collect_segments(seq_lens, batch, cap_len, lo, hi, b_start, p_start, list,
-                                           64, scratch, &more, &rb, &rp, &err);
+      int rb = batch, rp = 0, n;
+      if (first && warp_plan) {
+        if (threadIdx.x < 32) {
+          const int total = warp_plan_segments(wp, lo, hi, list, 64, &rb, &rp);
+          if (threadIdx.x == 0) {
+            words[0] = total;
+            words[1] = rb;
+            words[2] = rp;
+          }
+        }
+        __syncthreads();
+        n = min(words[0], 64);
+        more = words[0] > 64;
+        rb = words[1];
+        rp = words[2];
+      } else {
+        n = block_collect_segments(seq_lens, batch, cap_len, lo, hi, b_start, p_start, list, 64, scratch, &more,
+                                   &rb, &rp, &err);
+      }
+      first = false;
       if (threadIdx.x == 0) {
         for (int i = 0; i < n; ++i, ++written) {
           if (written >= max_segments) continue;

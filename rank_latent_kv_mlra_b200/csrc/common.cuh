@@ -140,6 +140,10 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 // ------------------------------------------------------------------------------------
 // Named barriers among a subset of warps
 // ------------------------------------------------------------------------------------
+// Arrives at named barrier `id` without waiting (the producer side of a hand-off).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -518,78 +522,109 @@ __device__ __forceinline__ int block_collect_segments(const int* __restrict__ se
   return count;
 }
 
-// One-pass planning for batches up to blockDim.x * kPlanPer sequences: each thread keeps the
-// lengths of its contiguous run of sequences in registers, so seq_lens is read once (one
-// memory round trip) instead of once per pass.
-constexpr int kPlanPer = 8;
-struct PlanRegs {
-  int n[kPlanPer];  // lengths (clamped) of sequences base .. base + per - 1
-  int base, per;
-  int first_p;      // flattened tile index where sequence `base` starts
-  int total;        // T = sum of tiles over all sequences
+constexpr int kPlanPer = 8;  // sequences per lane in the warp-level plan
+
+// Warp-level planning for batches up to 32 * kPlanPer sequences: every warp that needs the
+// plan computes it on its own (one read of seq_lens, a 5-step shuffle scan), with no block
+// barrier, so warps do not wait on one another. Lane l owns sequences [l*per, (l+1)*per).
+struct WarpPlan {
+  int n[kPlanPer];  // clamped lengths of the lane's sequences
+  int per, base;
+  int excl;         // flattened first tile of the lane's first sequence
+  int total;        // T = sum of tiles over all sequences (same in every lane)
 };
 
-// All threads call it. Returns false (and loads nothing) when the batch is too large for
-// the register plan; callers then use the multi-pass routines above.
-__device__ __forceinline__ bool block_plan_load(const int* __restrict__ seq_lens, int batch, int cap_len,
-                                                PlanRegs& pr, int* scratch, int* err) {
-  pr.per = (batch + blockDim.x - 1) / blockDim.x;
-  if (pr.per > kPlanPer) return false;
-  pr.base = threadIdx.x * pr.per;
+// All lanes call it. Returns false (and loads nothing) when the batch is too large.
+__device__ __forceinline__ bool warp_plan_load(const int* __restrict__ seq_lens, int batch, int cap_len,
+                                               WarpPlan& wp, int* err) {
+  wp.per = (batch + 31) / 32;
+  if (wp.per > kPlanPer) return false;
+  wp.base = lane_id() * wp.per;
   int local = 0;
 #pragma unroll
   for (int i = 0; i < kPlanPer; ++i) {
-    const int b = pr.base + i;
-    pr.n[i] = (i < pr.per && b < batch) ? clamp_len(__ldg(seq_lens + b), cap_len, err) : 0;
-    local += tiles_of(pr.n[i]);
+    const int b = wp.base + i;
+    wp.n[i] = (i < wp.per && b < batch) ? clamp_len(__ldg(seq_lens + b), cap_len, err) : 0;
+    local += tiles_of(wp.n[i]);
   }
-  pr.first_p = block_scan_tiles(local, scratch, &pr.total);
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane_id() >= o) incl += y;
+  }
+  wp.excl = incl - local;
+  wp.total = __shfl_sync(0xffffffffu, incl, 31);
   return true;
 }
 
-// Segments of the flattened tile range [lo, hi) from a register plan; same result and order
-// as block_collect_segments. Writes at most cap_list entries; returns the number of segments
-// in the range (which may exceed cap_list: then the caller resumes with the multi-pass
-// routine from (*resume_b, *resume_p)).
-__device__ __forceinline__ int block_plan_segments(const PlanRegs& pr, int lo, int hi, Segment* list, int cap_list,
-                                                   int* scratch, int* resume_b, int* resume_p) {
-  int hits = 0;
-  int pb = pr.first_p;
+// Flattened first tile of sequence b (warp-uniform, 0 <= b < batch) and its tile count.
+__device__ __forceinline__ int warp_plan_start(const WarpPlan& wp, int b, int* tiles) {
+  int before = wp.excl, t = 0;
 #pragma unroll
   for (int i = 0; i < kPlanPer; ++i) {
-    const int t = tiles_of(pr.n[i]);
-    if (i < pr.per && t > 0 && pb < hi && pb + t > lo) ++hits;
+    const int ti = tiles_of(wp.n[i]);
+    if (wp.base + i < b) before += ti;
+    if (wp.base + i == b) t = ti;
+  }
+  const int owner = b / wp.per;
+  *tiles = __shfl_sync(0xffffffffu, t, owner);
+  return __shfl_sync(0xffffffffu, before, owner);
+}
+
+// Segments of the flattened tile range [lo, hi) from a warp plan, in sequence order (the same
+// list block_plan_segments builds). One warp calls it. Writes at most cap_list entries and
+// returns how many segments the range holds; when that exceeds cap_list, (*resume_b,
+// *resume_p) name the first segment left out and its flattened start, for
+// block_collect_segments to continue from.
+__device__ __forceinline__ int warp_plan_segments(const WarpPlan& wp, int lo, int hi, Segment* list, int cap_list,
+                                                  int* resume_b, int* resume_p) {
+  int hits = 0;
+  int pb = wp.excl;
+#pragma unroll
+  for (int i = 0; i < kPlanPer; ++i) {
+    const int t = tiles_of(wp.n[i]);
+    if (i < wp.per && t > 0 && pb < hi && pb + t > lo) ++hits;
     pb += t;
   }
-  int total_hits;
-  int ord = block_scan_tiles(hits, scratch, &total_hits);
-  pb = pr.first_p;
+  int incl = hits;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane_id() >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int ord = incl - hits;
+  int res_b = 0, res_p = 0;
+  bool found = false;
+  pb = wp.excl;
 #pragma unroll
   for (int i = 0; i < kPlanPer; ++i) {
-    const int t = tiles_of(pr.n[i]);
-    if (i < pr.per && t > 0 && pb < hi && pb + t > lo) {
+    const int t = tiles_of(wp.n[i]);
+    if (i < wp.per && t > 0 && pb < hi && pb + t > lo) {
       if (ord < cap_list) {
         Segment sg;
-        sg.b = pr.base + i;
+        sg.b = wp.base + i;
         sg.tile_begin = max(lo, pb) - pb;
         sg.tile_end = min(hi, pb + t) - pb;
-        sg.n = pr.n[i];
+        sg.n = wp.n[i];
         list[ord] = sg;
       } else if (ord == cap_list) {
-        scratch[34] = pr.base + i;
-        scratch[35] = pb;
+        res_b = wp.base + i;
+        res_p = pb;
+        found = true;
       }
       ++ord;
     }
     pb += t;
   }
-  __syncthreads();
-  if (total_hits > cap_list) {
-    *resume_b = scratch[34];
-    *resume_p = scratch[35];
+  const unsigned m = __ballot_sync(0xffffffffu, found);
+  if (m) {
+    const int src = __ffs(m) - 1;
+    *resume_b = __shfl_sync(0xffffffffu, res_b, src);
+    *resume_p = __shfl_sync(0xffffffffu, res_p, src);
   }
-  __syncthreads();
-  return total_hits;
+  return total;
 }
 
 }  // namespace mlra

@@ -32,6 +32,7 @@
 namespace mlra {
 
 constexpr float kRescaleSlack = 8.0f;
+constexpr int kPlanBar = 5;  // named barrier of the segment-list hand-off (1..4: softmax groups)
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   volatile int* abort_flag = misc + 1;
   int* plan_err = misc + 2;
   int* scratch = misc + 8;  // 40 ints for the planner
+  volatile int* plan_words = misc + 48;  // segment count and resume point of the first list
 
   const int warp = warp_id(), lane = lane_id();
   const int group = blockIdx.x / p.nsub;
@@ -258,10 +260,12 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 
   // ---- plan: which flattened tiles this group owns (seq_lens do not depend on the
   // previous kernel, so this overlaps its tail under programmatic dependent launch) ----
+  // Batches up to 32 * kPlanPer: every warp scans seq_lens on its own (no block barrier) and
+  // warp 0 writes the segment list; larger batches use block-wide scans.
   int err = 0;
-  PlanRegs pr;
-  const bool reg_plan = block_plan_load(p.seq_lens, p.batch, cap_len, pr, scratch, &err);
-  const int T = reg_plan ? pr.total : block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
+  WarpPlan wp;
+  const bool warp_plan = warp_plan_load(p.seq_lens, p.batch, cap_len, wp, &err);
+  const int T = warp_plan ? wp.total : block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
   const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
   const int lo = min(group * quota, T);
   const int hi = min(lo + quota, T);
@@ -277,15 +281,38 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
   for (int x = 0; x < Sh::HW; ++x) l_part[x] = 0.f;
 
+  // first segment list from the warp plan: warp 0 builds it and hands it over through a
+  // named barrier, so it goes on to issue loads while the other warps pick the list up
+  int first_total = 0, first_rb = p.batch, first_rp = 0;
+  if (warp_plan && lo < hi) {
+    if (warp == 0) {
+      first_total = warp_plan_segments(wp, lo, hi, segs, Sh::MAX_SEGS, &first_rb, &first_rp);
+      if (lane == 0) {
+        plan_words[0] = first_total;
+        plan_words[1] = first_rb;
+        plan_words[2] = first_rp;
+      }
+      __threadfence_block();
+      __syncwarp();
+      named_bar_arrive(kPlanBar, Sh::THREADS);
+    } else {
+      named_bar_sync(kPlanBar, Sh::THREADS);
+      first_total = plan_words[0];
+      first_rb = plan_words[1];
+      first_rp = plan_words[2];
+    }
+  }
+
   int b_start = 0, p_start = 0;
   bool more = lo < hi;
   bool first_list = true;
   while (more) {
     int nseg, rb = p.batch, rp = 0;
-    if (first_list && reg_plan) {
-      const int total = block_plan_segments(pr, lo, hi, segs, Sh::MAX_SEGS, scratch, &rb, &rp);
-      nseg = min(total, Sh::MAX_SEGS);
-      more = total > Sh::MAX_SEGS;
+    if (first_list && warp_plan) {
+      nseg = min(first_total, Sh::MAX_SEGS);
+      more = first_total > Sh::MAX_SEGS;
+      rb = first_rb;
+      rp = first_rp;
     } else {
       int more_i;
       nseg = block_collect_segments(p.seq_lens, p.batch, cap_len, lo, hi, b_start, p_start, segs,

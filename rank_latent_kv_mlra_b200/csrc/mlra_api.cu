@@ -155,14 +155,16 @@ template <int DB, int DH, int NT>
 cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   using S = ProjShape<DB, DH, NT>;
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(128), S::SMEM1, s, false, &attr);
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, false,
+                                    &attr);
   return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, pp);
 }
 template <int DB, int DH, int NT, bool LATENT>
 cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   using S = ProjShape<DB, DH, NT>;
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(128), S::SMEM4, s, true, &attr);
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM4, s, true,
+                                    &attr);
   return cudaLaunchKernelEx(&c, mlra_uproj_kernel<S, LATENT>, h->map_wuv, pp);
 }
 template <int DB, int DH>
@@ -596,28 +598,6 @@ int mlra_test_decode_stalled(mlra_handle h, const void* q, mlra_dtype q_dtype, c
 #ifdef MLRA_TRACE
 // Profiling builds only: points the kernels' trace points at a device buffer of
 // [3 kernels][1024 CTAs][512 points] uint64 (NULL turns tracing off).
-// Profiling builds only: one launch of the absorb kernel alone (same arguments as a decode).
-int mlra_trace_absorb_only(mlra_handle h, const void* q, int batch, void* workspace, void* stream) {
-  Workspace w = carve(h, batch, workspace);
-  ProjParams pp = {};
-  pp.q = q;
-  pp.q_f32 = 0;
-  pp.q_pack = w.q_pack;
-  pp.qscale = h->scale * kLog2e;
-  pp.d_r = h->d_r;
-  pp.np = h->np;
-  pp.nsub = h->nsub;
-  pp.chunks = h->chunks;
-  pp.heads_block = h->heads_block;
-  pp.batch = batch;
-  pp.h = h->cfg.h;
-  pp.status = w.status;
-  pp.wait_limit_ns = kWaitLimitNs;
-  if (h->var != kMlra4) return MLRA_ERR_UNSUPPORTED;
-  return dispatch_absorb<128, 128>(h, pp, batch, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MLRA_OK
-                                                                                                   : MLRA_ERR_CUDA;
-}
-
 int mlra_trace_set(void* device_buffer) {
   return cudaMemcpyToSymbol(g_mlra_trace, &device_buffer, sizeof(device_buffer)) == cudaSuccess
              ? MLRA_OK

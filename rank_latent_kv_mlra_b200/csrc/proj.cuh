@@ -11,8 +11,9 @@
 // Both are one CTA per (head, batch tile): D^T[M x N] = A_h[M x K] * X_h[N x K]^T with the
 // per-head weight as the tcgen05 A operand (M = 128 rows of the weight's output dim; TMA
 // load) and the batch as N (16..128; filled by the CTA's threads, because the activation
-// side needs a dtype conversion or a merge on the way in). 128 threads: every warp reads one
-// TMEM lane quadrant in the epilogue.
+// side needs a dtype conversion or a merge on the way in). 512 threads: these kernels are
+// short chains of dependent steps, so four warps per scheduler hide each other's latencies;
+// in the epilogue warp w reads TMEM lane quadrant w % 4, column group w / 4.
 #pragma once
 
 #include "common.cuh"
@@ -21,6 +22,9 @@
 namespace mlra {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// threads of the combine / up-projection kernel: 16 warps, so the latency-bound merge and the
+// epilogue are spread over four warps per scheduler
+constexpr int kProjThreads = 512;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct ProjParams {
@@ -91,7 +95,7 @@ struct ProjShape {
 // absorb
 // ---------------------------------------------------------------------------------------
 template <class Sh>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kProjThreads, 1)
     mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -150,14 +154,14 @@ __global__ void __launch_bounds__(128, 1)
     const int qwh = DH + p.d_r;        // elements of one q row
     const int cpr = qwh / 8;           // chunks per row
     const int nch = NT * cpr;
-    constexpr int RND = 8;
+    constexpr int RND = 2;
     if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 10);
-    for (int base = 0; base < nch; base += 128 * RND) {
+    for (int base = 0; base < nch; base += kProjThreads * RND) {
       float v[RND][8];
       bool use[RND];
 #pragma unroll
       for (int i = 0; i < RND; ++i) {
-        const int idx = base + i * 128 + threadIdx.x;
+        const int idx = base + i * kProjThreads + threadIdx.x;
         const int bl = idx / cpr, d8 = (idx % cpr) * 8;
         const int b = n0 + bl;
         use[i] = idx < nch;
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int i = 0; i < RND; ++i) {
         if (!use[i]) continue;
-        const int idx = base + i * 128 + threadIdx.x;
+        const int idx = base + i * kProjThreads + threadIdx.x;
         const int bl = idx / cpr, d8 = (idx % cpr) * 8;
         if (d8 < DH) {
           uint4 w;
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(128, 1)
   // rows of a head chunk that no head fills (h/k below the MMA width) are zero
   if (hb == p.heads_block - 1 && prow == hb % p.np) {
     const int pad = p.np - 1 - prow;
-    for (int idx = threadIdx.x; idx < NT * pad * qw; idx += 128) {
+    for (int idx = threadIdx.x; idx < NT * pad * qw; idx += kProjThreads) {
       const int bl = idx / (pad * qw), rest = idx % (pad * qw);
       const int b = n0 + bl;
       if (b >= p.batch) continue;
@@ -254,25 +258,32 @@ __global__ void __launch_bounds__(128, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 4);
   if (ok) {
     // D^T (lanes = latent features, columns = batch rows) -> bf16 rows [b][c] in shared
-    // memory (the weight tile is no longer read), then 16-byte stores of whole rows.
-    tc_fence_after();
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    __nv_bfloat16* stage_out = reinterpret_cast<__nv_bfloat16*>(A);
+    // memory (the weight tile is no longer read), then 16-byte stores of whole rows. Warp w
+    // reads lane quadrant w % 4 (the quadrant its warp id may access) and column group w / 4.
+    constexpr int COLS = NT / 4 >= 8 ? NT / 4 : 8;
+    const int q4 = warp & 3, cg = warp >> 2;
+    if (cg * COLS < NT) {
+      tc_fence_after();
+      const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+      __nv_bfloat16* stage_out = reinterpret_cast<__nv_bfloat16*>(A);
 #pragma unroll
-    for (int mt = 0; mt < Sh::NMT; ++mt) {
-      const int c = mt * 128 + warp * 32 + lane;
-      float v[NT];
-      tmem_load_row<NT>(tbase + lane_base + mt * NT, v);
-      tmem_ld_wait();
-      if (c < DB) {
+      for (int mt = 0; mt < Sh::NMT; ++mt) {
+        const int c = mt * 128 + q4 * 32 + lane;
+        float v[COLS];
+        tmem_load_row<COLS>(tbase + lane_base + mt * NT + cg * COLS, v);
+        tmem_ld_wait();
+        if (c < DB) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) stage_out[n * DB + c] = __float2bfloat16_rn(v[n] * p.qscale);
+          for (int n = 0; n < COLS; ++n)
+            stage_out[(cg * COLS + n) * DB + c] = __float2bfloat16_rn(v[n] * p.qscale);
+        }
       }
     }
   }
+  tc_fence_before();
   __syncthreads();
   if (ok) {
-    for (int idx = threadIdx.x; idx < NT * (DB / 8); idx += 128) {
+    for (int idx = threadIdx.x; idx < NT * (DB / 8); idx += kProjThreads) {
       const int n = idx / (DB / 8), c8 = (idx % (DB / 8)) * 8;
       const int b = n0 + n;
       if (b < p.batch)
@@ -296,7 +307,7 @@ __global__ void __launch_bounds__(128, 1)
 // combine + uproj (LATENT_ONLY: combine and write o~ in fp32, no projection)
 // ---------------------------------------------------------------------------------------
 template <class Sh, bool LATENT_ONLY>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kProjThreads, 1)
     mlra_uproj_kernel(const __grid_constant__ CUtensorMap map_wuv, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -344,19 +355,15 @@ __global__ void __launch_bounds__(128, 1)
                     head * DB + r0, pol);
   }
 
-  // plan: total tiles and the flattened start of each sequence of this batch tile
+  // plan: total tiles, and where each sequence of this batch tile starts in the flattened
+  // tile order. Small batches: every warp computes it alone (no block barrier); large ones:
+  // a block-wide scan into pref[].
   int err = 0;
-  PlanRegs pr;
+  WarpPlan wp;
+  const bool warp_plan = warp_plan_load(p.seq_lens, p.batch, cap_len, wp, &err);
   int T;
-  if (block_plan_load(p.seq_lens, p.batch, cap_len, pr, scratch, &err)) {
-    T = pr.total;
-    int pb = pr.first_p;
-#pragma unroll
-    for (int i = 0; i < kPlanPer; ++i) {
-      const int b = pr.base + i;
-      if (i < pr.per && b >= n0 && b < n0 + NT) pref[b - n0] = pb;
-      pb += tiles_of(pr.n[i]);
-    }
+  if (warp_plan) {
+    T = wp.total;
   } else {
     T = block_total_tiles(p.seq_lens, p.batch, cap_len, scratch, &err);
     int running = 0;
@@ -368,23 +375,24 @@ __global__ void __launch_bounds__(128, 1)
       if (b >= n0 && b < n0 + NT) pref[b - n0] = pb;
       running += chunk_total;
     }
+    __syncthreads();
   }
   const int quota = T > 0 ? (T + p.groups - 1) / p.groups : 1;
   if (err) atomicOr(err_flag, 1);
-  __syncthreads();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 1);
 
   grid_dependency_wait();  // the partials come from the decode kernel
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 2);
 
   // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major).
-  // Each warp takes RB batch rows at a time and issues every load of a round (the rows'
-  // lse values and partial vectors, up to SB segments each) before using any of them, so a
-  // round costs one memory round trip. Rows with more segments take further rounds.
+  // Warp w takes batch rows w*RB .. w*RB+RB-1 (then + NW*RB ...) and issues every load of a
+  // round (the rows' lse values and partial vectors, up to SB segments each) before using
+  // any of them, so a round costs one memory round trip.
+  constexpr int NW = kProjThreads / 32;
   constexpr int PER = DB / 32;  // features per lane
-  constexpr int RB = 4;         // rows per warp per round
-  constexpr int SB = 4;         // segments per row loaded together
-  for (int r0 = warp * RB; r0 < NT; r0 += 4 * RB) {
+  constexpr int RB = 2;         // rows per warp per round
+  constexpr int SB = PER >= 8 ? 2 : 4;  // segments per row loaded together
+  for (int r0 = warp * RB; r0 < NT; r0 += NW * RB) {
     int c0[RB], nsg[RB];
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
@@ -392,9 +400,14 @@ __global__ void __launch_bounds__(128, 1)
       c0[rb] = 0;
       nsg[rb] = 0;
       if (bl < NT && b < p.batch) {
-        const int tb = tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err));
+        int tb, pb;
+        if (warp_plan) {
+          pb = warp_plan_start(wp, b, &tb);
+        } else {
+          tb = tiles_of(clamp_len(__ldg(p.seq_lens + b), cap_len, &err));
+          pb = pref[bl];
+        }
         if (tb > 0) {
-          const int pb = pref[bl];
           c0[rb] = pb / quota;
           nsg[rb] = (pb + tb - 1) / quota - c0[rb] + 1;
         }
@@ -412,6 +425,7 @@ __global__ void __launch_bounds__(128, 1)
     int maxseg = 0;
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) maxseg = max(maxseg, nsg[rb]);
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 7);
     for (int s0 = 0; s0 < maxseg; s0 += SB) {
       float lv[RB][SB];
       float v[RB][SB][PER];
@@ -462,6 +476,7 @@ __global__ void __launch_bounds__(128, 1)
         mx[rb] = m_new;
       }
     }
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 8);
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
       const int bl = r0 + rb, b = n0 + bl;
@@ -492,6 +507,7 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
     }
+    if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 9);
   }
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 3);
   if (err) atomicOr(err_flag, 1);
@@ -524,29 +540,35 @@ __global__ void __launch_bounds__(128, 1)
     if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 5);
     if (ok) {
       // D^T (lanes = head-dim d, columns = batch rows) -> rows [b][d] in shared memory (the
-      // operand tiles are no longer read), then 16-byte stores of whole output rows.
-      tc_fence_after();
-      const int d = warp * 32 + lane;
-      float v[NT];
-      tmem_load_row<NT>(tbase + (static_cast<uint32_t>(warp * 32) << 16), v);
-      tmem_ld_wait();
-      if (d < DH) {
-        if (p.out_f32) {
-          float* so = reinterpret_cast<float*>(A);
+      // operand tiles are no longer read), then 16-byte stores of whole output rows. Warp w
+      // reads lane quadrant w % 4 (the quadrant its warp id may access) and column group w / 4.
+      constexpr int COLS = NT / 4 >= 8 ? NT / 4 : 8;
+      const int q4 = warp & 3, cg = warp >> 2;
+      const int d = q4 * 32 + lane;
+      if (cg * COLS < NT) {
+        tc_fence_after();
+        float v[COLS];
+        tmem_load_row<COLS>(tbase + (static_cast<uint32_t>(q4 * 32) << 16) + cg * COLS, v);
+        tmem_ld_wait();
+        if (d < DH) {
+          if (p.out_f32) {
+            float* so = reinterpret_cast<float*>(A);
 #pragma unroll
-          for (int n = 0; n < NT; ++n) so[n * DH + d] = v[n];
-        } else {
-          __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(A);
+            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = v[c];
+          } else {
+            __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(A);
 #pragma unroll
-          for (int n = 0; n < NT; ++n) so[n * DH + d] = __float2bfloat16_rn(v[n]);
+            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = __float2bfloat16_rn(v[c]);
+          }
         }
       }
     }
+    tc_fence_before();
     __syncthreads();
     if (ok) {
       const int esz = p.out_f32 ? 4 : 2;
       const int chunks = DH * esz / 16;  // 16-byte pieces per output row
-      for (int idx = threadIdx.x; idx < NT * chunks; idx += 128) {
+      for (int idx = threadIdx.x; idx < NT * chunks; idx += kProjThreads) {
         const int n = idx / chunks, c = idx % chunks;
         const int b = n0 + n;
         if (b < p.batch)
