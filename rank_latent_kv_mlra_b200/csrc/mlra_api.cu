@@ -27,19 +27,29 @@ namespace {
 // Compiled kernel set. A variant fixes (d_b, d_rope, heads per CTA, d_h) and the decode
 // kernel's shared-memory pipeline.
 // ---------------------------------------------------------------------------------------
-enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kNumVariants };
+enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kNumVariants };
 
 using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 using DecMlra4 = DecodeShape<128, 64, 32, 4, 1, 2>;
 using DecMlra4q2 = DecodeShape<128, 64, 32, 3, 2, 2>;
 using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
+// MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits
+using DecMla = DecodeShape<512, 64, 32, 1, 1, 2>;
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 
 struct VariantDims {
   int d_b, d_r, np, d_h;
 };
-constexpr VariantDims kDims[kNumVariants] = {{32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}};
+constexpr VariantDims kDims[kNumVariants] = {
+    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 32, 128}};
+
+// Largest batch tile of the projection kernels: at d_b = 512 a 128-row tile of the merged
+// latent plus W^UV^T would need 256 KB of shared memory.
+template <int DB>
+constexpr int max_nt() {
+  return DB >= 512 ? 64 : 128;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -79,7 +89,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
-int nt_for(int batch) { return batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : 128; }
+int nt_for(int batch, int max_nt) {
+  const int nt = batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : 128;
+  return nt < max_nt ? nt : max_nt;
+}
 
 }  // namespace
 
@@ -127,7 +140,8 @@ cudaError_t prep_proj_all() {
   if ((e = prep_proj<DB, DH, 16>()) != cudaSuccess) return e;
   if ((e = prep_proj<DB, DH, 32>()) != cudaSuccess) return e;
   if ((e = prep_proj<DB, DH, 64>()) != cudaSuccess) return e;
-  return prep_proj<DB, DH, 128>();
+  if constexpr (max_nt<DB>() >= 128) return prep_proj<DB, DH, 128>();
+  return cudaSuccess;
 }
 
 // Programmatic dependent launch is on except inside a profiled call (thread-local, so a
@@ -169,20 +183,24 @@ cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cud
 }
 template <int DB, int DH>
 cudaError_t dispatch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
-  switch (nt_for(batch)) {
+  switch (nt_for(batch, max_nt<DB>())) {
     case 16: return launch_absorb<DB, DH, 16>(h, pp, batch, s);
     case 32: return launch_absorb<DB, DH, 32>(h, pp, batch, s);
     case 64: return launch_absorb<DB, DH, 64>(h, pp, batch, s);
-    default: return launch_absorb<DB, DH, 128>(h, pp, batch, s);
+    default:
+      if constexpr (max_nt<DB>() >= 128) return launch_absorb<DB, DH, 128>(h, pp, batch, s);
+      return cudaErrorInvalidValue;
   }
 }
 template <int DB, int DH, bool LATENT>
 cudaError_t dispatch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
-  switch (nt_for(batch)) {
+  switch (nt_for(batch, max_nt<DB>())) {
     case 16: return launch_uproj<DB, DH, 16, LATENT>(h, pp, batch, s);
     case 32: return launch_uproj<DB, DH, 32, LATENT>(h, pp, batch, s);
     case 64: return launch_uproj<DB, DH, 64, LATENT>(h, pp, batch, s);
-    default: return launch_uproj<DB, DH, 128, LATENT>(h, pp, batch, s);
+    default:
+      if constexpr (max_nt<DB>() >= 128) return launch_uproj<DB, DH, 128, LATENT>(h, pp, batch, s);
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -335,6 +353,15 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
         e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
                    : dispatch_uproj<256, 128, false>(h, pp, batch, s);
       break;
+    case kMla:
+      e = dispatch_absorb<512, 128>(h, pp, batch, s);
+      rec(1);
+      if (e == cudaSuccess) e = launch_decode<DecMla>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<512, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<512, 128, false>(h, pp, batch, s);
+      break;
     default:
       return MLRA_ERR_UNSUPPORTED;
   }
@@ -399,7 +426,9 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   const int d_b = c.d_c / c.k, hb = c.h / c.k;
   int var = -1;
   for (int v = 0; v < kNumVariants; ++v)
-    if (kDims[v].d_b == d_b && kDims[v].d_r == c.d_rope && kDims[v].d_h == c.d_h && hb <= kDims[v].np) var = v;
+    if (kDims[v].d_b == d_b && kDims[v].d_r == c.d_rope && kDims[v].d_h == c.d_h &&
+        (hb <= kDims[v].np || hb % kDims[v].np == 0))
+      var = v;
   if (var < 0) return MLRA_ERR_UNSUPPORTED;
 
   int dev = 0;
@@ -448,6 +477,11 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
       e = prep_decode<DecMlra2>();
       if (e == cudaSuccess) e = prep_proj_all<256, 128>();
       h->stages = DecMlra2::STAGES;
+      break;
+    case kMla:
+      e = prep_decode<DecMla>();
+      if (e == cudaSuccess) e = prep_proj_all<512, 128>();
+      h->stages = DecMla::STAGES;
       break;
     default:
       break;

@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   // any of them, so a round costs one memory round trip.
   constexpr int NW = kProjThreads / 32;
   constexpr int PER = DB / 32;  // features per lane
-  constexpr int RB = 2;         // rows per warp per round
+  constexpr int RB = PER >= 16 ? 1 : 2;  // rows per warp per round
   constexpr int SB = PER >= 8 ? 2 : 4;  // segments per row loaded together
   for (int r0 = warp * RB; r0 < NT; r0 += NW * RB) {
     int c0[RB], nsg[RB];

@@ -36,6 +36,7 @@ SMALL = {
     "mlra4_small": _small("mlra4_h128_b32_n8192", batch=3, seq_len=None, len_range=(1, 1500), seed=11),
     "mlra2_small": _small("mlra2_h128_b64_n4096", batch=3, seq_len=None, len_range=(100, 1300), seed=12),
     "mlra4_ragged_small": _small("mlra4_h128_b128_ragged1k_32k", batch=6, len_range=(1, 2000), seed=13),
+    "mla_small": _small("mla_h128_b128_ragged1k_32k", batch=5, len_range=(1, 1500), seed=14),
 }
 
 
@@ -88,10 +89,11 @@ def test_decode_output_matches_oracle(name, out_dtype):
                     tol_rel=1e-3)
 
 
-def test_split_partials_match_oracle():
+@pytest.mark.parametrize("name", ["mlra4_small", "mla_small"])
+def test_split_partials_match_oracle(name):
     """Every (segment, head) partial the decode kernel writes equals the oracle's partial
     over the same token range (the plan is checked bit-exact separately)."""
-    w = SMALL["mlra4_small"]
+    w = SMALL[name]
     inp = W.make_workload(w, device="cuda")
     hdl = G.make_handle(w, inp)
     _, _, ws = G.run_decode(hdl, inp, latent=True)
@@ -118,15 +120,16 @@ def test_split_partials_match_oracle():
     assert worst < 2e-2, worst
 
 
-@pytest.mark.parametrize("name", ["mlra4_small", "mlra2_small", "tiny_full"])
+@pytest.mark.parametrize("name", ["mlra4_small", "mlra2_small", "mla_small", "tiny_full"])
 def test_plan_is_bit_exact(name):
     w = SMALL[name]
     inp = W.make_workload(w, device="cuda")
     hdl = G.make_handle(w, inp)
     groups = M.mlra_get_info(hdl)["groups"]
     rng = np.random.default_rng(5)
+    # batches up to 256 take the warp-level plan, larger ones the block-wide scans
     cases = [inp["seq_lens"].cpu().tolist(), [0, 0, 5], [8192] * 32, list(rng.integers(0, 40000, 128)),
-             [1] * 300]
+             list(rng.integers(0, 3000, 256)), list(rng.integers(0, 3000, 257)), [1] * 300]
     for lens in cases:
         sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
         got, n = M.mlra_plan(hdl, sl, pt_stride=1024)
@@ -264,8 +267,6 @@ FULL = [n for n in W.WORKLOADS if n != "mlra4_h8_b1_n256_f32"]
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled(name):
     w = W.WORKLOADS[name]
-    if w.k == 1:
-        pytest.skip("k=1 (MLA) kernel set not compiled yet")
     inp = W.make_workload(w, device="cuda")
     hdl = G.make_handle(w, inp)
     out, lse, ws = G.run_decode(hdl, inp, out_dtype=torch.float32)
