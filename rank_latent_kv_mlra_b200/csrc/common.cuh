@@ -108,17 +108,19 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
 // Waits until the phase with the given parity of `bar` has completed. Gives up, raising the
 // CTA's abort flag, once `limit_ns` has passed or another role raised the flag. Returns false
 // when it gave up. Every wait in these kernels goes through here, so no wait is endless.
-// The wait polls (test_wait never suspends) with a short sleep between polls: a sleeping
-// warp leaves its issue slots to the warps sharing its scheduler, and wakes within ~0.1 us.
+// The wait is mbarrier.try_wait, which suspends the warp in hardware until the phase completes
+// (or a short hardware time limit passes), so a waiter wakes as soon as its data is there and
+// leaves its issue slots to the other warps meanwhile. The limit is counted in SM cycles at
+// kCyclesPerNs, i.e. at least `limit_ns` of wall time at clocks up to 2 GHz.
+constexpr uint64_t kCyclesPerNs = 2;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
-  if (mbar_poll(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = clock64();
   while (true) {
-    __nanosleep(32);
-    if (mbar_poll(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
+    if (clock64() - t0 > kCyclesPerNs * limit_ns) {
       *abort_flag = 1;
       return false;
     }
