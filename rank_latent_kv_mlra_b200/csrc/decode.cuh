@@ -15,10 +15,11 @@
 // Tokens sit on the MMA's M dimension because a block serves only h/k heads (32 for MLRA-4),
 // fewer than the 64/128 rows an MMA needs.
 //
-// Roles (64 + 128*NWG threads): warp 0 issues TMA loads of pages and queries, warp 1
-// allocates TMEM and issues the MMAs, warps 2.. form NWG softmax warpgroups (each owns a
-// slice of the heads) that run the softmax and write the partial results. They
-// hand off through mbarriers; each wait is bounded (see mbar_wait).
+// Roles (96 + 128*NWG threads): warp 0 issues TMA loads of pages and queries, warp 1
+// allocates TMEM and issues the QK MMAs, warps 2 .. 1+4*NWG form NWG softmax warpgroups (each
+// owns a slice of the heads) that run the softmax and write the partial results, and the last
+// warp issues the PV MMAs. Each issuer tracks its own MMAs with its own tcgen05.commit
+// barriers. The roles hand off through mbarriers; each wait is bounded (see mbar_wait).
 //
 // Softmax detail: each thread owns one token row of S^T and all its heads. The running
 // maximum m_h is only raised when some score exceeds it by more than kRescaleSlack (in
@@ -43,7 +44,8 @@ struct DecodeShape {
   static constexpr int NP = NP_;      // heads per CTA (MMA N), 16 / 32 / 64
   static constexpr int NWG = 2;       // softmax warpgroups; each owns NP / NWG heads
   static constexpr int HW = NP / NWG;
-  static constexpr int THREADS = 64 + 128 * NWG;
+  static constexpr int PV_WARP = 2 + 4 * NWG;  // after the softmax warps
+  static constexpr int THREADS = 32 * (PV_WARP + 1);
   static constexpr int STAGES = STAGES_;
   static constexpr int QBUF = QBUF_;  // query buffers
   static constexpr int PBUF = PBUF_;  // probability buffers
@@ -80,7 +82,7 @@ struct DecodeShape {
   static constexpr int OFF_RED = OFF_M + NP * 4;                // 4 x NP floats
   static constexpr int OFF_SEG = OFF_RED + 4 * NP * 4;          // MAX_SEGS segments
   static constexpr int OFF_BAR = round_up(OFF_SEG + MAX_SEGS * 16, 8);
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 8 + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 8 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, flags, scratch
   static constexpr int SMEM_BYTES = OFF_MISC + 64 * 4 + 1024;  // + alignment slack
   static_assert(DB % CW == 0 && DR % RW == 0, "region split");
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   uint64_t* sfree_bar = sfull_bar + 2;
   uint64_t* pfull_bar = sfree_bar + 2;
   uint64_t* pvdone_bar = pfull_bar + 2;
-  uint64_t* mmadone_bar = pvdone_bar + 2;
+  uint64_t* mmadone_bar = pvdone_bar + 2;  // [0] QK issuer, [1] PV issuer
   int* misc = reinterpret_cast<int*>(smem + Sh::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = misc + 1;
@@ -234,7 +236,8 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       mbar_init(&pfull_bar[s], 4 * Sh::NWG);
       mbar_init(&pvdone_bar[s], 1);
     }
-    mbar_init(mmadone_bar, 1);
+    mbar_init(&mmadone_bar[0], 1);
+    mbar_init(&mmadone_bar[1], 1);
     *abort_flag = 0;
     *plan_err = 0;
     fence_mbar_init();
@@ -403,46 +406,82 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
         }
       }
     } else if (warp == 1) {
-      // ============================== MMA issuer ==============================
-      // One thread issues. Two cursors walk the list's tiles: QK(i) needs tile i's pages
-      // (and, at a segment start, its query) plus a free S buffer; PV(i) needs P(i) from the
-      // softmax. Whichever is ready goes first, PV preferred: it releases a pipeline stage, so
-      // late page data never holds back a finished tile's PV and with it the next loads.
-      // Polling never suspends the thread, so neither condition waits behind the other.
+      // ============================== QK issuer ==============================
+      // One thread issues S^T(i) = [c_j | k^R](i) [q~ | q^R]^T once tile i's pages (and, at a
+      // segment start, its query) have landed and the softmax has read the S buffer's previous
+      // contents. The PVs have their own issuing warp, so a finished P never waits behind a
+      // QK wait here.
       if (lane == 0) {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NP, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NP, true, true);
-        struct Cursor {
-          int si, t;
-          uint32_t it, segc;
-        };
-        Cursor cq{0, nseg > 0 ? segs[0].tile_begin : 0, it, segc};
-        Cursor cp = cq;
-        uint32_t list_tiles = 0;
-        for (int i = 0; i < nseg; ++i) list_tiles += segs[i].tile_end - segs[i].tile_begin;
-        const uint32_t it_end = it + list_tiles;
-        auto advance = [&](Cursor& c) {
-          ++c.it;
-          if (++c.t == segs[c.si].tile_end) {
-            ++c.si;
-            ++c.segc;
-            if (c.si < nseg) c.t = segs[c.si].tile_begin;
-          }
-        };
-        bool q_ready = false;  // query of cq's segment has landed
-        uint64_t t_idle = 0;
-#ifdef MLRA_TRACE
-        uint32_t traced_arrival = 0xffffffffu;
-#endif
-        while (cp.it < it_end) {
-          bool issued = false;
-          if (cp.it < cq.it && mbar_poll(&pfull_bar[cp.it & 1], (cp.it >> 1) & 1)) {
-            // ---- PV(cp.it): O^T += C^T P^T
+        uint32_t ci = it, sc = segc;
+        bool ok = true;
+        for (int si = 0; si < nseg && ok; ++si) {
+          const Segment sg = segs[si];
+          const int qb = sc % Sh::QBUF;
+          ok = mbar_wait(&qfull_bar[qb], (sc / Sh::QBUF) & 1, abort_flag, p.wait_limit_ns);
+          for (int t = sg.tile_begin; t < sg.tile_end && ok; ++t, ++ci) {
+            ok = mbar_wait(&full_bar[ci % STAGES], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
+            if (ok && ci >= 2) ok = mbar_wait(&sfree_bar[ci & 1], ((ci >> 1) - 1) & 1, abort_flag, p.wait_limit_ns);
+            if (!ok) break;
             tc_fence_after();
-            MLRA_TRACE_POINT(1, 72 + min((int)cp.it, 31));
-            const bool first = cp.t == segs[cp.si].tile_begin;
-            const uint32_t st_addr = smem_u32(stages + (cp.it % STAGES) * Sh::STAGE_BYTES);
-            const uint32_t p_addr = smem_u32(pbufs + (cp.it % Sh::PBUF) * Sh::P_BYTES);
+            MLRA_TRACE_POINT(1, 40 + min((int)ci, 31));
+            const uint32_t st_addr = smem_u32(stages + (ci % STAGES) * Sh::STAGE_BYTES);
+            const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
+            const uint32_t d = tbase + Sh::S_COL0 + (ci & 1) * NP;
+            uint32_t acc = 0;
+#pragma unroll
+            for (int r = 0; r < Sh::NC; ++r) {
+#pragma unroll
+              for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
+                const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                             swizzle_code(Sh::C_ROWB));
+                const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                             swizzle_code(Sh::C_ROWB));
+                umma_bf16(d, a, b, idesc_qk, acc);
+                acc = 1;
+              }
+            }
+#pragma unroll
+            for (int r = 0; r < Sh::NR; ++r) {
+#pragma unroll
+              for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
+                const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
+                                             8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
+                                             8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                umma_bf16(d, a, b, idesc_qk, 1);
+              }
+            }
+            umma_commit(&sfull_bar[ci & 1]);
+            if (t == sg.tile_end - 1) umma_commit(&qempty_bar[qb]);
+          }
+          ++sc;
+        }
+        segc = sc;
+      }
+      __syncwarp();
+      uint32_t list_tiles = 0;
+      for (int i = 0; i < nseg; ++i) list_tiles += segs[i].tile_end - segs[i].tile_begin;
+      it += list_tiles;
+      segc = __shfl_sync(0xffffffffu, segc, 0);
+    } else if (warp == Sh::PV_WARP) {
+      // ============================== PV issuer ==============================
+      // One thread issues O^T += C_j^T(i) P^T(i) as soon as both softmax warpgroups have
+      // written P(i), then frees tile i's pipeline stage and signals pvdone.
+      if (lane == 0) {
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NP, true, true);
+        uint32_t pi = it;
+        bool ok = true;
+        for (int si = 0; si < nseg && ok; ++si) {
+          const Segment sg = segs[si];
+          for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++pi) {
+            ok = mbar_wait(&pfull_bar[pi & 1], (pi >> 1) & 1, abort_flag, p.wait_limit_ns);
+            if (!ok) break;
+            tc_fence_after();
+            MLRA_TRACE_POINT(1, 72 + min((int)pi, 31));
+            const bool first = t == sg.tile_begin;
+            const uint32_t st_addr = smem_u32(stages + (pi % STAGES) * Sh::STAGE_BYTES);
+            const uint32_t p_addr = smem_u32(pbufs + (pi % Sh::PBUF) * Sh::P_BYTES);
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
 #pragma unroll
@@ -454,84 +493,15 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                 umma_bf16(tbase + Sh::O_COL + mt * NP, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
               }
             }
-            umma_commit(&empty_bar[cp.it % STAGES]);
-            umma_commit(&pvdone_bar[cp.it & 1]);
-            advance(cp);
-            issued = true;
-          } else if (cq.it < it_end) {
-            const int qb = cq.segc % Sh::QBUF;
-            const bool seg_first = cq.t == segs[cq.si].tile_begin;
-            if (seg_first && !q_ready) q_ready = mbar_poll(&qfull_bar[qb], (cq.segc / Sh::QBUF) & 1);
-            const bool data = mbar_poll(&full_bar[cq.it % STAGES], (cq.it / STAGES) & 1);
-#ifdef MLRA_TRACE
-            if (data && cq.it != traced_arrival) {
-              traced_arrival = cq.it;
-              MLRA_TRACE_POINT(1, 232 + min((int)cq.it, 23));
-            }
-#endif
-            if ((!seg_first || q_ready) && data &&
-                (cq.it < 2 || mbar_poll(&sfree_bar[cq.it & 1], ((cq.it >> 1) - 1) & 1))) {
-              // ---- QK(cq.it): S^T = [c_j | k^R] [q~ | q^R]^T
-              tc_fence_after();
-              MLRA_TRACE_POINT(1, 40 + min((int)cq.it, 31));
-              const uint32_t st_addr = smem_u32(stages + (cq.it % STAGES) * Sh::STAGE_BYTES);
-              const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
-              const uint32_t d = tbase + Sh::S_COL0 + (cq.it & 1) * NP;
-              uint32_t acc = 0;
-#pragma unroll
-              for (int r = 0; r < Sh::NC; ++r) {
-#pragma unroll
-                for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
-                  const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                               swizzle_code(Sh::C_ROWB));
-                  const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                               swizzle_code(Sh::C_ROWB));
-                  umma_bf16(d, a, b, idesc_qk, acc);
-                  acc = 1;
-                }
-              }
-#pragma unroll
-              for (int r = 0; r < Sh::NR; ++r) {
-#pragma unroll
-                for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
-                  const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
-                                               8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                  const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
-                                               8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                  umma_bf16(d, a, b, idesc_qk, 1);
-                }
-              }
-              umma_commit(&sfull_bar[cq.it & 1]);
-              if (cq.t == segs[cq.si].tile_end - 1) {
-                umma_commit(&qempty_bar[qb]);
-                q_ready = false;
-              }
-              advance(cq);
-              issued = true;
-            }
-          }
-          if (issued) {
-            t_idle = 0;
-          } else {
-            // nothing ready: sleep briefly (leaves issue slots to the softmax warps on this
-            // scheduler), bounded like every other wait in this kernel
-            __nanosleep(32);
-            if (*abort_flag) break;
-            const uint64_t now = global_timer_ns();
-            if (t_idle == 0) {
-              t_idle = now;
-            } else if (now - t_idle > p.wait_limit_ns) {
-              *abort_flag = 1;
-              break;
-            }
+            umma_commit(&empty_bar[pi % STAGES]);
+            umma_commit(&pvdone_bar[pi & 1]);
           }
         }
-        it = it_end;
-        segc = cq.segc;
       }
       __syncwarp();
-      it = __shfl_sync(0xffffffffu, it, 0);
-      segc = __shfl_sync(0xffffffffu, segc, 0);
+      uint32_t list_tiles = 0;
+      for (int i = 0; i < nseg; ++i) list_tiles += segs[i].tile_end - segs[i].tile_begin;
+      it += list_tiles;
     } else {
       // ============================== softmax / epilogue ==============================
       // NWG warpgroups, each owning HW of the CTA's heads (S^T / O^T columns and P bytes of
@@ -723,10 +693,11 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       mbar_wait_drain(&full_bar[s], (last_it / STAGES) & 1, p.wait_limit_ns);
     }
   }
-  if (warp == 1) {
-    if (lane == 0) umma_commit(mmadone_bar);
+  if (warp == 1 || warp == Sh::PV_WARP) {
+    uint64_t* done = &mmadone_bar[warp == 1 ? 0 : 1];
+    if (lane == 0) umma_commit(done);
     __syncwarp();
-    mbar_wait_drain(mmadone_bar, 0, p.wait_limit_ns);
+    mbar_wait_drain(done, 0, p.wait_limit_ns);
   }
   tc_fence_before();
   __syncthreads();
