@@ -273,29 +273,59 @@ def run_ours(args, world, rank, local):
     k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kevs) / args.steps for i in range(3)]
     clk = clocks.stop()
 
-    # end to end through the public API: pinned host q and seq_lens in, output back to host
+    # End to end through the public API: every step uploads its query and lengths from pinned
+    # host memory and reads its output back into pinned host memory, inside the timed region.
+    # Steps are pipelined the way a serving loop runs them: uploads on one copy stream,
+    # downloads on another and two device buffer sets, so the copies of one step overlap the
+    # kernels of its neighbours (events order upload -> kernels -> download, and a buffer set is
+    # reused only after the step that last used it has finished with it).
+    NB = 2
     q_host = inp["q"].cpu().pin_memory()
     sl_host = inp["seq_lens"].cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    q_dev = torch.empty_like(inp["q"])
-    sl_dev = torch.empty_like(inp["seq_lens"])
-    e2e_args = (hdl, q_dev, inp["pool"], inp["page_table"], sl_dev, out)
-    for _ in range(max(3, args.warmup // 10)):
-        q_dev.copy_(q_host, non_blocking=True)
-        sl_dev.copy_(sl_host, non_blocking=True)
-        M.mlra_decode(*e2e_args, workspace=ws)
-        out_host.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(NB)]
+    q_dev = [torch.empty_like(inp["q"]) for _ in range(NB)]
+    sl_dev = [torch.empty_like(inp["seq_lens"]) for _ in range(NB)]
+    outs = [torch.empty_like(out) for _ in range(NB)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(NB)]
+    ev_dec = [torch.cuda.Event() for _ in range(NB)]
+    ev_down = [torch.cuda.Event() for _ in range(NB)]
+
+    def e2e_step(i):
+        k = i % NB
+        with torch.cuda.stream(up):
+            if i >= NB:
+                up.wait_event(ev_dec[k])  # the kernels of step i - NB have read q_dev[k]
+            q_dev[k].copy_(q_host, non_blocking=True)
+            sl_dev[k].copy_(sl_host, non_blocking=True)
+            ev_up[k].record(up)
+        stream.wait_event(ev_up[k])
+        if i >= NB:
+            stream.wait_event(ev_down[k])  # step i - NB's output has been read back
+        M.mlra_decode(hdl, q_dev[k], inp["pool"], inp["page_table"], sl_dev[k], outs[k], workspace=ws)
+        ev_dec[k].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_dec[k])
+            out_host[k].copy_(outs[k], non_blocking=True)
+            ev_down[k].record(down)
+
+    def e2e_run(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        up.wait_event(e0)
+        down.wait_event(e0)
+        for i in range(n):
+            e2e_step(i)
+        stream.wait_event(ev_down[(n - 1) % NB])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    e2e_run(max(3, args.warmup // 10))
     e2e_steps = max(10, args.steps // 4)
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        q_dev.copy_(q_host, non_blocking=True)
-        sl_dev.copy_(sl_host, non_blocking=True)
-        M.mlra_decode(*e2e_args, workspace=ws)
-        out_host.copy_(out, non_blocking=True)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    e2e_ms = e2e_run(e2e_steps)
+    # the pipelined steps computed the same output as the plain call
+    assert torch.equal(out_host[(e2e_steps - 1) % NB], out.cpu())
 
     step_ms_max = max_over_ranks(step_ms, world, dev)
     e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
@@ -324,7 +354,8 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": world * nbytes / (e2e_ms_max * 1e-3) / 1e9, "unit": UNIT,
                 "ms_per_step": e2e_ms_max,
                 "h2d_bytes_per_step": q_host.numel() * q_host.element_size() + sl_host.numel() * 4,
-                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+                "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
+                "pipelined": "uploads, kernels and downloads of consecutive steps overlap on three streams"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
@@ -345,7 +376,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
-    ap.add_argument("--cpu-pairs", type=int, default=400)
+    ap.add_argument("--cpu-pairs", type=int, default=6000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -421,7 +421,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           ok = mbar_wait(&qfull_bar[qb], (sc / Sh::QBUF) & 1, abort_flag, p.wait_limit_ns);
           for (int t = sg.tile_begin; t < sg.tile_end && ok; ++t, ++ci) {
             ok = mbar_wait(&full_bar[ci % STAGES], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
+            MLRA_TRACE_POINT(1, 400 + min((int)ci, 31));
             if (ok && ci >= 2) ok = mbar_wait(&sfree_bar[ci & 1], ((ci >> 1) - 1) & 1, abort_flag, p.wait_limit_ns);
+            MLRA_TRACE_POINT(1, 432 + min((int)ci, 31));
             if (!ok) break;
             tc_fence_after();
             MLRA_TRACE_POINT(1, 40 + min((int)ci, 31));
@@ -476,6 +478,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           const Segment sg = segs[si];
           for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++pi) {
             ok = mbar_wait(&pfull_bar[pi & 1], (pi >> 1) & 1, abort_flag, p.wait_limit_ns);
+            MLRA_TRACE_POINT(1, 464 + min((int)pi, 31));
             if (!ok) break;
             tc_fence_after();
             MLRA_TRACE_POINT(1, 72 + min((int)pi, 31));

@@ -89,6 +89,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over the query [batch][heads][cols]: box = cols x 1 head x box_b batch rows,
+// landing as box_b rows of box_cols in shared memory.
+bool make_q_map(CUtensorMap* m, const void* q, uint64_t batch, uint64_t heads, uint64_t cols, uint32_t box_cols,
+                uint32_t box_b, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, heads, batch};
+  cuuint64_t strides[2] = {cols * 2, heads * cols * 2};
+  cuuint32_t box[3] = {box_cols, 1, box_b};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int nt_for(int batch, int max_nt) {
   const int nt = batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 64 ? 64 : 128;
   return nt < max_nt ? nt : max_nt;
@@ -168,10 +183,21 @@ cudaLaunchConfig_t launch_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s
 template <int DB, int DH, int NT>
 cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   using S = ProjShape<DB, DH, NT>;
+  // a bf16 query is read by TMA: its q^C columns in swizzle-width boxes, its q^R columns in one
+  // unswizzled box
+  CUtensorMap mqc, mqr;
+  std::memset(&mqc, 0, sizeof(mqc));
+  std::memset(&mqr, 0, sizeof(mqr));
+  if (!pp.q_f32) {
+    const uint64_t cols = (uint64_t)DH + h->d_r;
+    if (!make_q_map(&mqc, pp.q, batch, h->cfg.h, cols, S::AW, NT, swizzle_for(S::AROWB)) ||
+        !make_q_map(&mqr, pp.q, batch, h->cfg.h, cols, h->d_r, NT, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
   cudaLaunchAttribute attr;
   cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, false,
                                     &attr);
-  return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, pp);
+  return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, mqc, mqr, pp);
 }
 template <int DB, int DH, int NT, bool LATENT>
 cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {

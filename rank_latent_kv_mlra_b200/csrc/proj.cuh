@@ -67,9 +67,13 @@ struct ProjShape {
   static constexpr int B1_REG = round_up(NT * AROWB, 1024);
   static constexpr int A1_BOXR = NMT * 128 < 256 ? NMT * 128 : 256;
   static constexpr int A1_TX = NKR * NMT * 128 * AROWB;
+  // q^R rows of the batch tile (bf16 query: loaded by TMA, then scaled into the packed query);
+  // room for d_rope up to 64
+  static constexpr int OFF_QRS = NKR * A1_REG + NKR * B1_REG;
+  static constexpr int QRS_BYTES = round_up(NT * 64 * 2, 1024);
   // operand tiles, reused afterwards to stage the output rows
-  static constexpr int STG1 = round_up(NKR * A1_REG + NKR * B1_REG > NT * DB * 2 ? NKR * A1_REG + NKR * B1_REG
-                                                                                  : NT * DB * 2, 1024);
+  static constexpr int STG1 = round_up(OFF_QRS + QRS_BYTES > NT * DB * 2 ? OFF_QRS + QRS_BYTES : NT * DB * 2, 1024);
+  static_assert(NT * DB * 2 <= OFF_QRS, "output staging must not overlap the q^R staging");
   static constexpr int SMEM1 = STG1 + 1024 + 256;
   static constexpr int TMEM1 = NMT * NT <= 32 ? 32 : NMT * NT <= 64 ? 64 : NMT * NT <= 128 ? 128 :
                                NMT * NT <= 256 ? 256 : 512;
@@ -96,7 +100,8 @@ struct ProjShape {
 // ---------------------------------------------------------------------------------------
 template <class Sh>
 __global__ void __launch_bounds__(kProjThreads, 1)
-    mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const ProjParams p) {
+    mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_qc,
+                       const __grid_constant__ CUtensorMap map_qr, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -118,11 +123,25 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 0);
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.status) *p.status = 0;
+  // a bf16 query comes in by TMA with the weight: [batch tile][q^C columns] straight into the
+  // MMA's swizzled B layout, [batch tile][q^R] into a staging tile (rows past the batch read 0)
+  const bool tma_q = !p.q_f32;
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // issue the loads first: nothing below depends on them until the MMA
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_arrive_expect_tx(&bars[0], Sh::A1_TX + (tma_q ? NT * (DH + p.d_r) * 2 : 0));
+    for (int kr = 0; kr < Sh::NKR; ++kr)
+      for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
+        tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW, head * DB + r0, pol);
+    if (tma_q) {
+      for (int kr = 0; kr < Sh::NKR; ++kr)
+        tma_load_3d(Bq + kr * Sh::B1_REG, &map_qc, &bars[0], kr * Sh::AW, head, n0, pol);
+      tma_load_3d(smem + Sh::OFF_QRS, &map_qr, &bars[0], DH, head, n0, pol);
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, Sh::TMEM1);
@@ -137,20 +156,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   // split planning now; they wait for this grid's results before reading them
   grid_launch_dependents();
 
-  if (threadIdx.x == 0) {
-    tma_prefetch_map(&map_wuk);
-    mbar_arrive_expect_tx(&bars[0], Sh::A1_TX);
-    const uint64_t pol = l2_policy_evict_first();
-    for (int kr = 0; kr < Sh::NKR; ++kr)
-      for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
-        tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW,
-                    head * DB + r0, pol);
-  }
-
   // q_h for the batch tile, in 8-element chunks: q^C chunks -> bf16, K-major swizzled tile
   // (the MMA's B operand); q^R chunks -> packed query, scaled. All global loads of a round are
   // issued before any store, so the round costs one memory round trip.
-  {
+  if (!tma_q) {
     const int qwh = DH + p.d_r;        // elements of one q row
     const int cpr = qwh / 8;           // chunks per row
     const int nch = NT * cpr;
@@ -252,6 +261,33 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         umma_commit(&bars[1]);
       }
       __syncwarp();
+    }
+  }
+  if (tma_q && warp != 0) {
+    // q^R from the staging tile, scaled, into the packed query (while warp 0 runs the MMA)
+    if (mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns)) {
+      const int cpr = p.d_r / 8;
+      const __nv_bfloat16* qrs = reinterpret_cast<const __nv_bfloat16*>(smem + Sh::OFF_QRS);
+      for (int idx = threadIdx.x - 32; idx < NT * cpr; idx += kProjThreads - 32) {
+        const int bl = idx / cpr, c8 = (idx % cpr) * 8;
+        const int b = n0 + bl;
+        if (b >= p.batch) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(qrs + bl * p.d_r + c8);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = __bfloat1622float2(h2[e]);
+          f[2 * e] = v.x * p.qscale;
+          f[2 * e + 1] = v.y * p.qscale;
+        }
+        uint4 w;
+        w.x = pack_bf16x2(f[0], f[1]);
+        w.y = pack_bf16x2(f[2], f[3]);
+        w.z = pack_bf16x2(f[4], f[5]);
+        w.w = pack_bf16x2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(p.q_pack + (((size_t)b * p.nsub + sub) * p.np + prow) * qw + DB + c8) = w;
+      }
     }
   }
   const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
