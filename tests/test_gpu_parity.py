@@ -282,3 +282,24 @@ def test_full_size_sampled(name):
     got_l = np.array([float(lse[b, hd]) for b, hd in pairs])
     exp_l = np.array([ref[p][2] for p in pairs])
     assert np.abs(got_l - exp_l).max() < G.TOL_LSE_ABS
+
+
+def test_bounded_wait_times_out_cleanly():
+    """A decode whose producer withholds every CTA's first tile: the consumer's pipeline wait
+    runs out after the given limit, every role drains and leaves, the status word reads
+    MLRA_ERR_TIMEOUT, and the context stays usable for the next call."""
+    import time
+    w = SMALL["mlra4_small"]
+    inp = W.make_workload(w, device="cuda")
+    hdl = G.make_handle(w, inp)
+    out = torch.zeros(w.batch, w.h, w.d_h, device="cuda")
+    ws = M.alloc_workspace(hdl, w.batch)
+    t0 = time.time()
+    M.mlra_test_decode_stalled(hdl, inp["q"], inp["pool"], inp["page_table"], inp["seq_lens"], out, ws,
+                               wait_limit_ns=2_000_000)
+    torch.cuda.synchronize()
+    assert M.mlra_get_status(ws) == -5  # MLRA_ERR_TIMEOUT
+    assert time.time() - t0 < 10
+    got, _, ws2 = G.run_decode(hdl, inp)
+    assert M.mlra_get_status(ws2) == 0
+    G.assert_parity(got.cpu().numpy(), G.oracle_full(w, inp)["out"], "decode after a timed-out call")
