@@ -398,7 +398,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
-    ap.add_argument("--cpu-pairs", type=int, default=6000)
+    ap.add_argument("--cpu-pairs", type=int, default=15000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
