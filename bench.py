@@ -52,10 +52,15 @@ def measured_hbm_peak():
 
 
 def kernel_source_hash():
+    """Hash of the decode kernel's code (comments and blank lines left out, so a comment edit
+    does not invalidate a recorded ncu capture)."""
     h = hashlib.sha256()
     for f in ["common.cuh", "decode.cuh"]:
-        with open(os.path.join(ROOT, "rank_latent_kv_mlra_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "rank_latent_kv_mlra_b200", "csrc", f), encoding="utf-8") as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

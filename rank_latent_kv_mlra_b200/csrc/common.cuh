@@ -92,7 +92,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test (never suspends the thread), for polling several barriers in turn.
+// Non-blocking test (never suspends the thread); the teardown drain polls with it.
 __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -584,7 +584,7 @@ __device__ __forceinline__ int warp_plan_start(const WarpPlan& wp, int b, int* t
 }
 
 // Segments of the flattened tile range [lo, hi) from a warp plan, in sequence order (the same
-// list block_plan_segments builds). One warp calls it. Writes at most cap_list entries and
+// list block_collect_segments builds). One warp calls it. Writes at most cap_list entries and
 // returns how many segments the range holds; when that exceeds cap_list, (*resume_b,
 // *resume_p) name the first segment left out and its flattened start, for
 // block_collect_segments to continue from.

@@ -31,7 +31,6 @@ enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kNumVariants };
 
 using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 using DecMlra4 = DecodeShape<128, 64, 32, 4, 1, 2>;
-using DecMlra4q2 = DecodeShape<128, 64, 32, 3, 2, 2>;
 using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
 // MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits
 using DecMla = DecodeShape<512, 64, 32, 1, 1, 2>;
@@ -363,8 +362,7 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
       e = dispatch_absorb<128, 128>(h, pp, batch, s);
       rec(1);
       if (e == cudaSuccess)
-        e = h->stages == 3 ? launch_decode<DecMlra4q2>(h, mc, mr, mqc, mqr, dp, s)
-                           : launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
+        e = launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
       rec(2);
       if (e == cudaSuccess)
         e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
@@ -489,15 +487,8 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
       break;
     case kMlra4:
       e = prep_decode<DecMlra4>();
-      if (e == cudaSuccess) e = prep_decode<DecMlra4q2>();
       if (e == cudaSuccess) e = prep_proj_all<128, 128>();
       h->stages = DecMlra4::STAGES;
-      {
-        // tuning switch: MLRA_DECODE_STAGES=3 selects the 3-stage pipeline with two query
-        // buffers (no bubble at segment changes) instead of 4 stages with one
-        const char* env = std::getenv("MLRA_DECODE_STAGES");
-        if (env != nullptr && std::atoi(env) == DecMlra4q2::STAGES) h->stages = DecMlra4q2::STAGES;
-      }
       break;
     case kMlra2:
       e = prep_decode<DecMlra2>();
