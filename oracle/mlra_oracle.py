@@ -32,9 +32,10 @@ Readings where the pages are silent (each is listed in the design doc):
 * k^R is one vector per token, shared by every head and block, cached already rotated;
 * every head has its own q^R_h; RoPE is applied upstream.
 
-Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` except
-``plan_segments``, whose rule is this build's own (the pages have no split-KV scheme); it is
-pinned by hand-worked golden cases and by invariants (coverage, disjointness, quota).
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (the
+summed-blocks functions by ``tests/test_oracle_summed.py``) except ``plan_segments``, whose rule
+is this build's own (the pages have no split-KV scheme); it is pinned by hand-worked golden
+cases and by invariants (coverage, disjointness, quota).
 """
 from __future__ import annotations
 
@@ -160,6 +161,92 @@ def decode_heads(q, w_uk, w_uv, rows, seq_heads, k, d_r, scale=None):
         lats.append(lat)
         lses.append(l)
     return np.array(outs), np.array(lats), np.array(lses)
+
+
+# ---------------------------------------------------------------------------------------
+# Summed-blocks reading: every head attends to every latent block with its own pair of
+# matrices per block, each block under its own softmax, and the head's output is the sum of
+# the k per-block outputs times alpha_attn. This is the reading that the MLRA index page's
+# Table 2 (MLRA-4: 4nh(d_c/4) + 2nh d_h^R FLOPs per device, all h heads on each device's
+# block) and the alpha_attn column of its model tables (Table 16: alpha_attn = 1/2 for
+# MLRA-2) point to; the partitioned reading above is the default one.
+# ---------------------------------------------------------------------------------------
+
+def default_attn_scale(k: int) -> float:
+    """alpha_attn when none is given: 1/k (the only value the pages print is 1/2 at k = 2)."""
+    return 1.0 / k
+
+
+def decode_summed(q, w_uk, w_uv, pool, page_table, seq_lens, k, d_r, scale=None, attn_scale=None,
+                  form="absorbed"):
+    """Full decode step under the summed-blocks reading.
+
+    q: [B][h][d_h + d_r]; w_uk, w_uv: [k][h][d_b][d_h]; the rest as in ``decode``.
+    ``out[b][h] = attn_scale * sum_j W^UV_{j,h} softmax_t(s_{j,h,t}) c_j[t]`` with
+    ``s_{j,h,t} = scale * (q^C_h . W^UK_{j,h} c_j[t] + q^R_h . k^R[t])``.
+    Returns ``out`` [B][h][d_h], ``lse`` [B][k][h] (each block's softmax, natural log) and, for
+    the absorbed form, ``latent`` [B][k][h][d_b]. An empty sequence gives zeros and lse = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w_uk = np.asarray(w_uk, dtype=np.float64)
+    w_uv = np.asarray(w_uv, dtype=np.float64)
+    pool = np.asarray(pool, dtype=np.float64)
+    B, h, qw = q.shape
+    d_h = qw - d_r
+    d_b = w_uk.shape[2]
+    d_c = d_b * k
+    if scale is None:
+        scale = default_scale(d_h, d_r)
+    if attn_scale is None:
+        attn_scale = default_attn_scale(k)
+    out = np.zeros((B, h, d_h))
+    lse = np.full((B, k, h), -np.inf)
+    latent = np.zeros((B, k, h, d_b))
+    for b in range(B):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        rows = gather_rows(pool, page_table, b, n)
+        for j in range(k):
+            c_j, kr = _split(rows, j, d_c, k)
+            for hd in range(h):
+                qc, qr = q[b, hd, :d_h], q[b, hd, d_h:]
+                if form == "explicit":
+                    o, lse[b, j, hd] = attend_head_explicit(qc, qr, w_uk[j, hd], w_uv[j, hd], c_j, kr, scale)
+                else:
+                    o, latent[b, j, hd], lse[b, j, hd] = attend_head_absorbed(
+                        qc, qr, w_uk[j, hd], w_uv[j, hd], c_j, kr, scale)
+                out[b, hd] += attn_scale * o
+    res = {"out": out, "lse": lse}
+    if form != "explicit":
+        res["latent"] = latent
+    return res
+
+
+def decode_summed_heads(q, w_uk, w_uv, rows, seq_heads, k, d_r, scale=None, attn_scale=None):
+    """``decode_summed`` for a list of heads of ONE sequence whose rows are given (sampled
+    checks at full size). Returns (out [len][d_h], lse [len][k])."""
+    q = np.asarray(q, dtype=np.float64)
+    w_uk = np.asarray(w_uk, dtype=np.float64)
+    w_uv = np.asarray(w_uv, dtype=np.float64)
+    d_b = w_uk.shape[2]
+    d_c = d_b * k
+    d_h = q.shape[-1] - d_r
+    if scale is None:
+        scale = default_scale(d_h, d_r)
+    if attn_scale is None:
+        attn_scale = default_attn_scale(k)
+    outs, lses = [], []
+    for hd in seq_heads:
+        o_sum = np.zeros(d_h)
+        l = np.zeros(k)
+        for j in range(k):
+            c_j, kr = _split(rows, j, d_c, k)
+            o, _, l[j] = attend_head_absorbed(q[hd, :d_h], q[hd, d_h:], w_uk[j, hd], w_uv[j, hd], c_j, kr, scale)
+            o_sum += attn_scale * o
+        outs.append(o_sum)
+        lses.append(l)
+    return np.array(outs), np.array(lses)
 
 
 # ---------------------------------------------------------------------------------------

@@ -49,6 +49,7 @@ class Workload:
     paging: str = "permuted"               # "permuted" | "contiguous"
     tiny_scaling: bool = False             # activations / sqrt(width)
     q_dtype: str = "bf16"                  # "bf16" | "f32"
+    summed: bool = False                   # every head attends to every block; outputs summed
 
     @property
     def d_b(self) -> int:
@@ -71,6 +72,9 @@ WORKLOADS = {
                  batch=128, len_range=(1024, 32768), seed=4),
         Workload("mla_h128_b128_ragged1k_32k", k=1, h=128, d_h=128, d_c=512, d_r=64,
                  batch=128, len_range=(1024, 32768), seed=4),
+        # the summed-blocks reading of MLRA-4 on the headline's shapes
+        Workload("mlra4sum_h128_b32_n8192", k=4, h=128, d_h=128, d_c=512, d_r=64, batch=32,
+                 seq_len=8192, seed=5, summed=True),
     ]
 }
 
@@ -165,8 +169,10 @@ def make_workload(w: Workload, device="cpu", seq_lens: Optional[torch.Tensor] = 
     q32[..., :w.d_h] *= qc_scale
     q32[..., w.d_h:] *= qr_scale
     w_scale = 1.0 / math.sqrt(d_b)
-    w_uk32 = randn(w.h, d_b, w.d_h) * w_scale
-    w_uv32 = randn(w.h, d_b, w.d_h) * w_scale
+    # [h][d_b][d_h], or [k][h][d_b][d_h] (one pair of matrices per block and head) when summed
+    wshape = (w.k, w.h, d_b, w.d_h) if w.summed else (w.h, d_b, w.d_h)
+    w_uk32 = randn(*wshape) * w_scale
+    w_uv32 = randn(*wshape) * w_scale
 
     out = {
         "workload": w,
