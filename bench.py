@@ -192,7 +192,10 @@ def oracle_sample_rate(w, inp, pairs_per_step, steps, warmup):
         for _ in range(pairs_per_step):
             b = int(rng.integers(0, w.batch))
             hd = int(rng.integers(0, w.h))
-            O.decode_heads(q[b], wuk, wuv, rows_of(b), [hd], w.k, w.d_r)
+            if w.summed:
+                O.decode_summed_heads(q[b], wuk, wuv, rows_of(b), [hd], w.k, w.d_r)
+            else:
+                O.decode_heads(q[b], wuk, wuv, rows_of(b), [hd], w.k, w.d_r)
 
     for _ in range(warmup):
         step()
@@ -219,7 +222,8 @@ def run_reference(args, world, rank):
         "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
-                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64},
+                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64,
+                   "reading": "summed" if w.summed else "partitioned"},
         "cpu_baseline": {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": "each step: the float64 oracle on one random (sequence, head) pair "
                                    f"of the {w.name} workload; value scaled by the fraction of the "
@@ -240,7 +244,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     w = W.WORKLOADS[args.workload]
     inp = W.make_workload(w, device=dev)
-    hdl = M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"])
+    hdl = M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed)
     B = w.batch
     out = torch.empty(B, w.h, w.d_h, device=dev, dtype=torch.bfloat16)
     ws = M.alloc_workspace(hdl, B, dev)
@@ -370,6 +374,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded; inputs larger than L2: the 302 MB cache stream evicts the 126 MB L2 each step)",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
                    "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
+                   "reading": "summed" if w.summed else "partitioned",
                    "l2": "inputs larger than L2", "parallelism": f"replicas{world}",
                    "cache_bytes_per_step": nbytes},
         "kernels_ms": {"absorb": k_ms[0], "decode": k_ms[1], "combine_uproj": k_ms[2]},
@@ -387,7 +392,8 @@ def run_ours(args, world, rank, local):
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
-        pairs = max(1, args.cpu_pairs)
+        # a summed-blocks head attends to all k blocks: k times the oracle work per pair
+        pairs = max(1, args.cpu_pairs // (w.k if w.summed else 1))
         rate, sec, threads = oracle_sample_rate(w, inp, pairs, 1, 0)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"float64 oracle on {pairs} random (sequence, head) pairs of "

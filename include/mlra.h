@@ -64,16 +64,29 @@ typedef struct {
   int k;               /* latent blocks; 1 = MLA. k must divide d_c and h */
   int page_size;       /* tokens per cache page; must be 64 */
   float softmax_scale; /* <= 0 selects 1/sqrt(d_h + d_rope) (a reading: the pages fix none) */
+  int blocks_summed;   /* 0: head group j = heads [j*h/k, (j+1)*h/k) attends only to block c_j
+                          (the default reading). 1: every head attends to every block with its
+                          own W^UK_{j,h}, W^UV_{j,h}, each block under its own softmax, and
+                          o_h = attn_scale * sum_j W^UV_{j,h} o~_{j,h} (the reading Table 2 and
+                          the alpha_attn entries of the MLRA index page's model tables point
+                          to). Weights are then [k][h][d_b][d_h] and lse is [batch][k*h],
+                          block-major (entry j*h + head). */
+  float attn_scale;    /* alpha_attn when blocks_summed: <= 0 selects 1/k (Table 16 prints 1/2
+                          for k = 2; a reading). Ignored otherwise. */
 } mlra_config;
 
-/* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, h/k, d_h):
- *   (32, 16, <=16, 32), (128, 64, <=32, 128), (256, 64, <=64, 128); batch <= 4096. */
+/* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, heads per block, d_h),
+ * heads per block being h/k, or h when blocks_summed:
+ *   (32, 16, <=16, 32), (128, 64, <=32 or a multiple of 32, 128),
+ *   (256, 64, <=64 or a multiple of 64, 128), (512, 64, a multiple of 32, 128) [k = 1, MLA];
+ * blocks_summed with (32, 16, ...) and (128, 64, ...) only; batch <= 4096. */
 
 typedef struct mlra_ctx* mlra_handle;
 
 /* Creates a handle. w_uk, w_uv: device bf16 [h][d_c/k][d_h], row-major: W^UK_h maps a
  * block latent to a key by K_h[d] = sum_c c[c] * w_uk[h][c][d] (the ai360xpert code's
  * (H, d_c, d_head) convention restricted to the head's block); likewise w_uv for values.
+ * With blocks_summed they are [k][h][d_c/k][d_h], one pair of matrices per block and head.
  * Borrowed, must stay valid and unchanged until mlra_destroy. *out receives the handle. */
 int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra_handle* out);
 

@@ -48,7 +48,8 @@ class MlraError(RuntimeError):
 class mlra_config(ctypes.Structure):
     _fields_ = [("h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_c", ctypes.c_int),
                 ("d_rope", ctypes.c_int), ("k", ctypes.c_int), ("page_size", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("blocks_summed", ctypes.c_int),
+                ("attn_scale", ctypes.c_float)]
 
 
 class mlra_info(ctypes.Structure):
@@ -136,13 +137,17 @@ class Handle:
 
 
 def mlra_create(h: int, d_h: int, d_c: int, d_rope: int, k: int, w_uk: torch.Tensor,
-                w_uv: torch.Tensor, softmax_scale: float = 0.0, page_size: int = 64) -> Handle:
+                w_uv: torch.Tensor, softmax_scale: float = 0.0, page_size: int = 64,
+                blocks_summed: bool = False, attn_scale: float = 0.0) -> Handle:
+    """blocks_summed: every head attends to every block with weights [k][h][d_c/k][d_h] and the
+    per-block outputs are summed times attn_scale (<= 0: 1/k); lse is then [batch][k*h]."""
     lib = load_library()
+    shape = (k, h, d_c // k, d_h) if blocks_summed else (h, d_c // k, d_h)
     for t, n in ((w_uk, "w_uk"), (w_uv, "w_uv")):
         _require(t, n, torch.bfloat16)
-        if tuple(t.shape) != (h, d_c // k, d_h):
-            raise ValueError(f"{n} must be [h][d_c/k][d_h]")
-    cfg = mlra_config(h, d_h, d_c, d_rope, k, page_size, softmax_scale)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{n} must be {'[k][h]' if blocks_summed else '[h]'}[d_c/k][d_h]")
+    cfg = mlra_config(h, d_h, d_c, d_rope, k, page_size, softmax_scale, int(blocks_summed), attn_scale)
     out = ctypes.c_void_p()
     _check(lib.mlra_create(ctypes.byref(cfg), _ptr(w_uk), _ptr(w_uv), ctypes.byref(out)), "mlra_create")
     return Handle(out, cfg, w_uk, w_uv)

@@ -118,6 +118,9 @@ struct mlra_ctx {
   int num_sms;
   Variant var;
   int d_b, d_r, np, chunks, nsub, heads_block, groups, stages;
+  int vh;         // heads of the packed query and partials: h, or k*h when the blocks are summed
+  bool summed;    // every head attends to every block; outputs summed
+  float alpha;    // alpha_attn (summed blocks)
   float scale;
   CUtensorMap map_wuk;
   CUtensorMap map_wuv;
@@ -147,6 +150,23 @@ cudaError_t prep_proj() {
   e = prep_kernel(mlra_uproj_kernel<S, false>, S::SMEM4);
   if (e != cudaSuccess) return e;
   return prep_kernel(mlra_uproj_kernel<S, true>, S::SMEM4);
+}
+// combine + up-projection over SUMK summed blocks
+template <int DB, int DH, int SUMK>
+cudaError_t prep_proj_sum() {
+  cudaError_t e;
+  if ((e = prep_kernel(mlra_uproj_kernel<ProjShape<DB, DH, 16>, false, SUMK>, ProjShape<DB, DH, 16>::SMEM4)) !=
+      cudaSuccess)
+    return e;
+  if ((e = prep_kernel(mlra_uproj_kernel<ProjShape<DB, DH, 32>, false, SUMK>, ProjShape<DB, DH, 32>::SMEM4)) !=
+      cudaSuccess)
+    return e;
+  if ((e = prep_kernel(mlra_uproj_kernel<ProjShape<DB, DH, 64>, false, SUMK>, ProjShape<DB, DH, 64>::SMEM4)) !=
+      cudaSuccess)
+    return e;
+  if constexpr (max_nt<DB>() >= 128)
+    return prep_kernel(mlra_uproj_kernel<ProjShape<DB, DH, 128>, false, SUMK>, ProjShape<DB, DH, 128>::SMEM4);
+  return cudaSuccess;
 }
 template <int DB, int DH>
 cudaError_t prep_proj_all() {
@@ -194,17 +214,19 @@ cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cu
       return cudaErrorInvalidValue;
   }
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, false,
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->vh, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, false,
                                     &attr);
   return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, mqc, mqr, pp);
 }
-template <int DB, int DH, int NT, bool LATENT>
+template <int DB, int DH, int NT, bool LATENT, int SUMK = 1>
 cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   using S = ProjShape<DB, DH, NT>;
+  // one CTA per output head; per virtual head when only the latent is wanted
+  const int gx = SUMK > 1 ? h->cfg.h : h->vh;
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->cfg.h, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM4, s, true,
+  cudaLaunchConfig_t c = launch_cfg(dim3(gx, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM4, s, true,
                                     &attr);
-  return cudaLaunchKernelEx(&c, mlra_uproj_kernel<S, LATENT>, h->map_wuv, pp);
+  return cudaLaunchKernelEx(&c, mlra_uproj_kernel<S, LATENT, SUMK>, h->map_wuv, pp);
 }
 template <int DB, int DH>
 cudaError_t dispatch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
@@ -217,14 +239,14 @@ cudaError_t dispatch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, 
       return cudaErrorInvalidValue;
   }
 }
-template <int DB, int DH, bool LATENT>
+template <int DB, int DH, bool LATENT, int SUMK = 1>
 cudaError_t dispatch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   switch (nt_for(batch, max_nt<DB>())) {
-    case 16: return launch_uproj<DB, DH, 16, LATENT>(h, pp, batch, s);
-    case 32: return launch_uproj<DB, DH, 32, LATENT>(h, pp, batch, s);
-    case 64: return launch_uproj<DB, DH, 64, LATENT>(h, pp, batch, s);
+    case 16: return launch_uproj<DB, DH, 16, LATENT, SUMK>(h, pp, batch, s);
+    case 32: return launch_uproj<DB, DH, 32, LATENT, SUMK>(h, pp, batch, s);
+    case 64: return launch_uproj<DB, DH, 64, LATENT, SUMK>(h, pp, batch, s);
     default:
-      if constexpr (max_nt<DB>() >= 128) return launch_uproj<DB, DH, 128, LATENT>(h, pp, batch, s);
+      if constexpr (max_nt<DB>() >= 128) return launch_uproj<DB, DH, 128, LATENT, SUMK>(h, pp, batch, s);
       return cudaErrorInvalidValue;
   }
 }
@@ -258,9 +280,9 @@ Workspace carve(const mlra_ctx* h, int batch, void* base) {
   off += align256((size_t)batch * h->nsub * h->np * (h->d_b + h->d_r) * 2);
   const size_t slots = (size_t)batch + h->groups;
   w.o_part = reinterpret_cast<float*>(p + off);
-  off += align256(slots * h->cfg.h * h->d_b * 4);
+  off += align256(slots * h->vh * h->d_b * 4);
   w.lse_part = reinterpret_cast<float*>(p + off);
-  off += align256(slots * h->cfg.h * 4);
+  off += align256(slots * h->vh * 4);
   w.bytes = off;
   return w;
 }
@@ -317,7 +339,10 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   pp.pt_stride = pt_stride;
   pp.groups = h->groups;
   pp.batch = batch;
-  pp.h = h->cfg.h;
+  pp.h = h->vh;
+  pp.q_heads = h->cfg.h;
+  pp.out_heads = h->cfg.h;
+  pp.out_scale = h->summed ? h->alpha : 1.f;
   pp.status = w.status;
   pp.wait_limit_ns = wait_limit_ns;
 
@@ -331,7 +356,7 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   dp.nsub = h->nsub;
   dp.chunks = h->chunks;
   dp.heads_block = h->heads_block;
-  dp.h = h->cfg.h;
+  dp.h = h->vh;
   dp.d_c = h->cfg.d_c;
   dp.o_part = w.o_part;
   dp.lse_part = w.lse_part;
@@ -356,7 +381,9 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
       if (e == cudaSuccess) e = launch_decode<DecTiny>(h, mc, mr, mqc, mqr, dp, s);
       rec(2);
       if (e == cudaSuccess)
-        e = latent ? dispatch_uproj<32, 32, true>(h, pp, batch, s) : dispatch_uproj<32, 32, false>(h, pp, batch, s);
+        e = latent      ? dispatch_uproj<32, 32, true>(h, pp, batch, s)
+            : h->summed ? dispatch_uproj<128, 32, false, 4>(h, pp, batch, s)
+                        : dispatch_uproj<32, 32, false>(h, pp, batch, s);
       break;
     case kMlra4:
       e = dispatch_absorb<128, 128>(h, pp, batch, s);
@@ -365,8 +392,9 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
         e = launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
       rec(2);
       if (e == cudaSuccess)
-        e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
-                   : dispatch_uproj<128, 128, false>(h, pp, batch, s);
+        e = latent      ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
+            : h->summed ? dispatch_uproj<512, 128, false, 4>(h, pp, batch, s)
+                        : dispatch_uproj<128, 128, false>(h, pp, batch, s);
       break;
     case kMlra2:
       e = dispatch_absorb<256, 128>(h, pp, batch, s);
@@ -447,13 +475,18 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   if (c.d_c % c.k != 0 || c.h % c.k != 0) return MLRA_ERR_INVALID_ARG;
   if (c.page_size != kPage) return MLRA_ERR_UNSUPPORTED;
   if (!aligned16(w_uk) || !aligned16(w_uv)) return MLRA_ERR_INVALID_ARG;
-  const int d_b = c.d_c / c.k, hb = c.h / c.k;
+  if (c.blocks_summed != 0 && c.blocks_summed != 1) return MLRA_ERR_INVALID_ARG;
+  const bool summed = c.blocks_summed == 1;
+  // heads per block: a group of h/k, or all h when every head attends to every block
+  const int d_b = c.d_c / c.k, hb = summed ? c.h : c.h / c.k;
   int var = -1;
   for (int v = 0; v < kNumVariants; ++v)
     if (kDims[v].d_b == d_b && kDims[v].d_r == c.d_rope && kDims[v].d_h == c.d_h &&
         (hb <= kDims[v].np || hb % kDims[v].np == 0))
       var = v;
   if (var < 0) return MLRA_ERR_UNSUPPORTED;
+  // summed blocks: the combine's GEMM runs over k*d_b, compiled for these two shapes
+  if (summed && !((var == kMlra4 && c.k == 4) || (var == kTiny && c.k == 4))) return MLRA_ERR_UNSUPPORTED;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLRA_ERR_CUDA;
@@ -472,6 +505,9 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   h->d_r = c.d_rope;
   h->np = kDims[var].np;
   h->heads_block = hb;
+  h->summed = summed;
+  h->vh = summed ? c.k * c.h : c.h;
+  h->alpha = c.attn_scale > 0.f ? c.attn_scale : 1.0f / (float)c.k;
   h->chunks = (hb + h->np - 1) / h->np;
   h->nsub = c.k * h->chunks;
   h->groups = h->num_sms / h->nsub;
@@ -483,11 +519,13 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
     case kTiny:
       e = prep_decode<DecTiny>();
       if (e == cudaSuccess) e = prep_proj_all<32, 32>();
+      if (e == cudaSuccess && summed) e = prep_proj_sum<128, 32, 4>();
       h->stages = DecTiny::STAGES;
       break;
     case kMlra4:
       e = prep_decode<DecMlra4>();
       if (e == cudaSuccess) e = prep_proj_all<128, 128>();
+      if (e == cudaSuccess && summed) e = prep_proj_sum<512, 128, 4>();
       h->stages = DecMlra4::STAGES;
       break;
     case kMlra2:
@@ -507,13 +545,13 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
     delete h;
     return MLRA_ERR_CUDA;
   }
-  // weight tensor maps: [h * d_b rows][d_h cols]
   const int aw = c.d_h < 64 ? c.d_h : 64;
   const int nmt_rows = d_b >= 128 ? d_b : 128;
   const uint32_t boxr1 = nmt_rows < 256 ? nmt_rows : 256;
   const uint32_t boxr4 = d_b < 256 ? d_b : 256;
-  if (!make_map(&h->map_wuk, w_uk, (uint64_t)c.h * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr1, aw) ||
-      !make_map(&h->map_wuv, w_uv, (uint64_t)c.h * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr4, aw)) {
+  // weight tensor maps: [vh * d_b rows][d_h cols], one d_b-row matrix per (virtual) head
+  if (!make_map(&h->map_wuk, w_uk, (uint64_t)h->vh * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr1, aw) ||
+      !make_map(&h->map_wuv, w_uv, (uint64_t)h->vh * d_b, c.d_h, (uint64_t)c.d_h * 2, boxr4, aw)) {
     delete h;
     return MLRA_ERR_CUDA;
   }

@@ -50,7 +50,11 @@ struct ProjParams {
   int groups;
   // common
   int batch;
-  int h;
+  int h;              // heads of the packed query and the partials (k*h virtual heads when the
+                      // blocks are summed)
+  int q_heads;        // heads of the query rows (head v reads query row v % q_heads)
+  int out_heads;      // heads of the output rows
+  float out_scale;    // alpha_attn when the blocks are summed, else 1
   int* status;
   unsigned long long wait_limit_ns;
 };
@@ -73,7 +77,6 @@ struct ProjShape {
   static constexpr int QRS_BYTES = round_up(NT * 64 * 2, 1024);
   // operand tiles, reused afterwards to stage the output rows
   static constexpr int STG1 = round_up(OFF_QRS + QRS_BYTES > NT * DB * 2 ? OFF_QRS + QRS_BYTES : NT * DB * 2, 1024);
-  static_assert(NT * DB * 2 <= OFF_QRS, "output staging must not overlap the q^R staging");
   static constexpr int SMEM1 = STG1 + 1024 + 256;
   static constexpr int TMEM1 = NMT * NT <= 32 ? 32 : NMT * NT <= 64 ? 64 : NMT * NT <= 128 ? 128 :
                                NMT * NT <= 256 ? 256 : 512;
@@ -103,6 +106,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_qc,
                        const __grid_constant__ CUtensorMap map_qr, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
+  static_assert(NT * DB * 2 <= Sh::OFF_QRS, "output staging must not overlap the q^R staging");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -138,9 +142,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
         tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW, head * DB + r0, pol);
     if (tma_q) {
+      const int qh = head % p.q_heads;
       for (int kr = 0; kr < Sh::NKR; ++kr)
-        tma_load_3d(Bq + kr * Sh::B1_REG, &map_qc, &bars[0], kr * Sh::AW, head, n0, pol);
-      tma_load_3d(smem + Sh::OFF_QRS, &map_qr, &bars[0], DH, head, n0, pol);
+        tma_load_3d(Bq + kr * Sh::B1_REG, &map_qc, &bars[0], kr * Sh::AW, qh, n0, pol);
+      tma_load_3d(smem + Sh::OFF_QRS, &map_qr, &bars[0], DH, qh, n0, pol);
     }
   }
   if (warp == 0) {
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int b = n0 + bl;
         use[i] = idx < nch;
         if (use[i] && b < p.batch) {
-          const size_t off = ((size_t)b * p.h + head) * qwh + d8;
+          const size_t off = ((size_t)b * p.q_heads + head % p.q_heads) * qwh + d8;
           if (p.q_f32) {
             const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.q) + off);
             const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
@@ -342,7 +347,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 // ---------------------------------------------------------------------------------------
 // combine + uproj (LATENT_ONLY: combine and write o~ in fp32, no projection)
 // ---------------------------------------------------------------------------------------
-template <class Sh, bool LATENT_ONLY>
+// SUMK > 1 (summed blocks): the CTA of output head `head` merges the partials of its SUMK
+// virtual heads j*out_heads + head (latent block j), lays them side by side along K
+// (DB = SUMK * block width) and multiplies by the SUMK stacked W^UV matrices in one GEMM, so
+// the sum over blocks happens in the tensor core's accumulator; out_scale applies alpha_attn.
+template <class Sh, bool LATENT_ONLY, int SUMK = 1>
 __global__ void __launch_bounds__(kProjThreads, 1)
     mlra_uproj_kernel(const __grid_constant__ CUtensorMap map_wuv, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
@@ -385,10 +394,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     tma_prefetch_map(&map_wuv);
     mbar_arrive_expect_tx(&bars[0], Sh::A4_TX);
     const uint64_t pol = l2_policy_evict_first();
+    constexpr int DBB = DB / SUMK;  // rows of one block's W^UV
+    constexpr int BOXR = DBB < Sh::A4_BOXR ? DBB : Sh::A4_BOXR;
     for (int a = 0; a < Sh::NATOM; ++a)
-      for (int r0 = 0; r0 < DB; r0 += Sh::A4_BOXR)
-        tma_load_2d(A + a * Sh::ATOM + r0 * Sh::AROWB, &map_wuv, &bars[0], a * Sh::AW,
-                    head * DB + r0, pol);
+      for (int j = 0; j < SUMK; ++j)
+        for (int r0 = 0; r0 < DBB; r0 += BOXR)
+          tma_load_2d(A + a * Sh::ATOM + (j * DBB + r0) * Sh::AROWB, &map_wuv, &bars[0], a * Sh::AW,
+                      (j * p.out_heads + head) * DBB + r0, pol);
   }
 
   // plan: total tiles, and where each sequence of this batch tile starts in the flattened
@@ -426,6 +438,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   // any of them, so a round costs one memory round trip.
   constexpr int NW = kProjThreads / 32;
   constexpr int PER = DB / 32;  // features per lane
+  constexpr int DBB = DB / SUMK;  // features of one block
+  static_assert(DBB % PER == 0, "a lane's features lie in one block");
+  // the (virtual) head whose partials this lane merges, and the lane's first feature in it
+  const int vhead = SUMK == 1 ? head : ((lane * PER) / DBB) * p.out_heads + head;
+  const int f0 = (lane * PER) % DBB;
   constexpr int RB = PER >= 16 ? 1 : 2;  // rows per warp per round
   constexpr int SB = PER >= 8 ? 2 : 4;  // segments per row loaded together
   for (int r0 = warp * RB; r0 < NT; r0 += NW * RB) {
@@ -472,8 +489,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int si = 0; si < SB; ++si) {
           if (s0 + si < nsg[rb]) {
             const size_t slot = (size_t)(b + c0[rb] + s0 + si);
-            lv[rb][si] = __ldg(p.lse_part + slot * p.h + head);
-            const float* src = p.o_part + (slot * p.h + head) * DB + lane * PER;
+            lv[rb][si] = __ldg(p.lse_part + slot * p.h + vhead);
+            const float* src = p.o_part + (slot * p.h + vhead) * DBB + f0;
             if constexpr (PER % 4 == 0) {
 #pragma unroll
               for (int e = 0; e < PER; e += 4) {
@@ -520,8 +537,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const float inv = sum[rb] > 0.f ? 1.f / sum[rb] : 0.f;
 #pragma unroll
       for (int e = 0; e < PER; ++e) acc[rb][e] *= inv;
-      if (b < p.batch && lane == 0 && p.lse_out)
-        p.lse_out[(size_t)b * p.h + head] = nsg[rb] > 0 ? (mx[rb] + log2f(sum[rb])) * kLn2 : -INFINITY;
+      if (b < p.batch && f0 == 0 && p.lse_out)  // one lane per (virtual) head
+        p.lse_out[(size_t)b * p.h + vhead] = nsg[rb] > 0 ? (mx[rb] + log2f(sum[rb])) * kLn2 : -INFINITY;
       if constexpr (LATENT_ONLY) {
         if (b < p.batch) {
           float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
@@ -590,11 +607,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           if (p.out_f32) {
             float* so = reinterpret_cast<float*>(A);
 #pragma unroll
-            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = v[c];
+            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = v[c] * p.out_scale;
           } else {
             __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(A);
 #pragma unroll
-            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = __float2bfloat16_rn(v[c]);
+            for (int c = 0; c < COLS; ++c) so[(cg * COLS + c) * DH + d] = __float2bfloat16_rn(v[c] * p.out_scale);
           }
         }
       }
@@ -608,7 +625,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int n = idx / chunks, c = idx % chunks;
         const int b = n0 + n;
         if (b < p.batch)
-          *reinterpret_cast<uint4*>(static_cast<char*>(p.out) + (((size_t)b * p.h + head) * DH) * esz + c * 16) =
+          *reinterpret_cast<uint4*>(static_cast<char*>(p.out) + (((size_t)b * p.out_heads + head) * DH) * esz + c * 16) =
               *reinterpret_cast<const uint4*>(A + (size_t)n * DH * esz + c * 16);
       }
     }
