@@ -37,7 +37,7 @@ constexpr int kPlanBar = 5;  // named barrier of the segment-list hand-off (1..4
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_>
+template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2>
 struct DecodeShape {
   static constexpr int DB = DB_;      // latent block width d_c / k
   static constexpr int DR = DR_;      // RoPE key width
@@ -48,7 +48,16 @@ struct DecodeShape {
   static constexpr int THREADS = 32 * (PV_WARP + 1);
   static constexpr int STAGES = STAGES_;
   static constexpr int QBUF = QBUF_;  // query buffers
-  static constexpr int PBUF = PBUF_;  // probability buffers
+  // probability buffers; 0: P(i) is written over the RoPE columns of tile i's own stage,
+  // which QK(i) has finished reading when the softmax sees S(i), and the stage is only
+  // reloaded after PV(i) has read it
+  static constexpr int PBUF = PBUF_;
+  static constexpr bool P_IN_STAGE = PBUF == 0;
+  // Depth of the P-ready / PV-done barrier rings. Tile i's softmax can only run once PV(i -
+  // STAGES) has freed tile i's stage, so with at least STAGES slots no ring slot is armed again
+  // before the phase it held has been waited for (no parity aliasing), however far the softmax
+  // runs ahead of the PV issuer.
+  static constexpr int PR = STAGES > 2 ? STAGES : 2;
   // A cache row is split into swizzle-width regions: block columns and RoPE columns.
   static constexpr int CW = DB < 64 ? DB : 64;
   static constexpr int NC = DB / CW;
@@ -68,9 +77,10 @@ struct DecodeShape {
   static constexpr int P_BYTES = round_up(kTile * P_ROWB, 1024);
   static constexpr int NMT = DB >= 128 ? DB / 128 : 1;  // PV M tiles
   static constexpr uint32_t PV_LBO = DB >= 128 ? C_REG : 0;  // next 64-feature chunk
-  static constexpr int S_COL0 = 0;                  // two S buffers of NP columns
-  static constexpr int O_COL = 2 * NP;              // NMT x NP columns
-  static constexpr int TMEM_USED = 2 * NP + NMT * NP;
+  static constexpr int SBUF = SBUF_;                // S buffers of NP columns in TMEM
+  static constexpr int S_COL0 = 0;
+  static constexpr int O_COL = SBUF * NP;           // NMT x NP columns
+  static constexpr int TMEM_USED = SBUF * NP + NMT * NP;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int MAX_SEGS = 64;
@@ -82,13 +92,15 @@ struct DecodeShape {
   static constexpr int OFF_RED = OFF_M + NP * 4;                // 4 x NP floats
   static constexpr int OFF_SEG = OFF_RED + 4 * NP * 4;          // MAX_SEGS segments
   static constexpr int OFF_BAR = round_up(OFF_SEG + MAX_SEGS * 16, 8);
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 8 + 2;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 2 * SBUF + 2 * PR + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, flags, scratch
   static constexpr int SMEM_BYTES = OFF_MISC + 64 * 4 + 1024;  // + alignment slack
   static_assert(DB % CW == 0 && DR % RW == 0, "region split");
   static_assert(NP == 16 || NP == 32 || NP == 64, "heads per CTA");
   static_assert(QBUF == 1 || QBUF == 2, "query buffers");
-  static_assert(PBUF == 1 || PBUF == 2, "P buffers");
+  static_assert(SBUF >= 2 && TMEM_USED <= 512, "S buffers");
+  static_assert(PBUF == 0 || PBUF == 1 || PBUF == 2, "P buffers");
+  static_assert(PBUF != 0 || P_BYTES <= NR * R_REG, "P must fit the RoPE region of a stage");
 };
 
 struct DecodeParams {
@@ -200,10 +212,10 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   uint64_t* qfull_bar = bars + 2 * STAGES;
   uint64_t* qempty_bar = qfull_bar + Sh::QBUF;
   uint64_t* sfull_bar = qempty_bar + Sh::QBUF;
-  uint64_t* sfree_bar = sfull_bar + 2;
-  uint64_t* pfull_bar = sfree_bar + 2;
-  uint64_t* pvdone_bar = pfull_bar + 2;
-  uint64_t* mmadone_bar = pvdone_bar + 2;  // [0] QK issuer, [1] PV issuer
+  uint64_t* sfree_bar = sfull_bar + Sh::SBUF;
+  uint64_t* pfull_bar = sfree_bar + Sh::SBUF;
+  uint64_t* pvdone_bar = pfull_bar + Sh::PR;
+  uint64_t* mmadone_bar = pvdone_bar + Sh::PR;  // [0] QK issuer, [1] PV issuer
   int* misc = reinterpret_cast<int*>(smem + Sh::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = misc + 1;
@@ -230,9 +242,11 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       mbar_init(&qfull_bar[s], 1);
       mbar_init(&qempty_bar[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Sh::SBUF; ++s) {
       mbar_init(&sfull_bar[s], 1);
       mbar_init(&sfree_bar[s], 4 * Sh::NWG);
+    }
+    for (int s = 0; s < Sh::PR; ++s) {
       mbar_init(&pfull_bar[s], 4 * Sh::NWG);
       mbar_init(&pvdone_bar[s], 1);
     }
@@ -422,14 +436,15 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           for (int t = sg.tile_begin; t < sg.tile_end && ok; ++t, ++ci) {
             ok = mbar_wait(&full_bar[ci % STAGES], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
             MLRA_TRACE_POINT(1, 400 + min((int)ci, 31));
-            if (ok && ci >= 2) ok = mbar_wait(&sfree_bar[ci & 1], ((ci >> 1) - 1) & 1, abort_flag, p.wait_limit_ns);
+            if (ok && ci >= Sh::SBUF)
+              ok = mbar_wait(&sfree_bar[ci % Sh::SBUF], ((ci / Sh::SBUF) - 1) & 1, abort_flag, p.wait_limit_ns);
             MLRA_TRACE_POINT(1, 432 + min((int)ci, 31));
             if (!ok) break;
             tc_fence_after();
             MLRA_TRACE_POINT(1, 40 + min((int)ci, 31));
             const uint32_t st_addr = smem_u32(stages + (ci % STAGES) * Sh::STAGE_BYTES);
             const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
-            const uint32_t d = tbase + Sh::S_COL0 + (ci & 1) * NP;
+            const uint32_t d = tbase + Sh::S_COL0 + (ci % Sh::SBUF) * NP;
             uint32_t acc = 0;
 #pragma unroll
             for (int r = 0; r < Sh::NC; ++r) {
@@ -454,7 +469,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                 umma_bf16(d, a, b, idesc_qk, 1);
               }
             }
-            umma_commit(&sfull_bar[ci & 1]);
+            umma_commit(&sfull_bar[ci % Sh::SBUF]);
             if (t == sg.tile_end - 1) umma_commit(&qempty_bar[qb]);
           }
           ++sc;
@@ -477,14 +492,15 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
         for (int si = 0; si < nseg && ok; ++si) {
           const Segment sg = segs[si];
           for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++pi) {
-            ok = mbar_wait(&pfull_bar[pi & 1], (pi >> 1) & 1, abort_flag, p.wait_limit_ns);
+            ok = mbar_wait(&pfull_bar[pi % Sh::PR], (pi / Sh::PR) & 1, abort_flag, p.wait_limit_ns);
             MLRA_TRACE_POINT(1, 464 + min((int)pi, 31));
             if (!ok) break;
             tc_fence_after();
             MLRA_TRACE_POINT(1, 72 + min((int)pi, 31));
             const bool first = t == sg.tile_begin;
             const uint32_t st_addr = smem_u32(stages + (pi % STAGES) * Sh::STAGE_BYTES);
-            const uint32_t p_addr = smem_u32(pbufs + (pi % Sh::PBUF) * Sh::P_BYTES);
+            const uint32_t p_addr = Sh::P_IN_STAGE ? st_addr + Sh::NC * Sh::C_REG
+                                                   : smem_u32(pbufs + (pi % max(Sh::PBUF, 1)) * Sh::P_BYTES);
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
 #pragma unroll
@@ -497,7 +513,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
               }
             }
             umma_commit(&empty_bar[pi % STAGES]);
-            umma_commit(&pvdone_bar[pi & 1]);
+            umma_commit(&pvdone_bar[pi % Sh::PR]);
           }
         }
       }
@@ -532,20 +548,20 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           const bool last = (t == sg.tile_end - 1);
           const bool tile_full = (t + 1) * kTile <= sg.n;
           const bool valid = t * kTile + row < sg.n;
-          bool okl = mbar_wait(&sfull_bar[it & 1], (it >> 1) & 1, abort_flag, p.wait_limit_ns);
-          if (it >= Sh::PBUF) {  // the PV that last read this P buffer must be done
+          bool okl = mbar_wait(&sfull_bar[it % Sh::SBUF], (it / Sh::SBUF) & 1, abort_flag, p.wait_limit_ns);
+          if (!Sh::P_IN_STAGE && it >= Sh::PBUF) {  // the PV that last read this P buffer must be done
             const uint32_t j = it - Sh::PBUF;
-            okl = okl && mbar_wait(&pvdone_bar[j & 1], (j >> 1) & 1, abort_flag, p.wait_limit_ns);
+            okl = okl && mbar_wait(&pvdone_bar[j % Sh::PR], (j / Sh::PR) & 1, abort_flag, p.wait_limit_ns);
           }
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 104 + min((int)it, 31));
           if (warp == 6 && lane == 0) MLRA_TRACE_POINT(1, 320 + min((int)it, 31));
           tc_fence_after();
           float s[HW];
-          tmem_load_row<HW>(tbase + lane_base + Sh::S_COL0 + (it & 1) * NP + hcol, s);
+          tmem_load_row<HW>(tbase + lane_base + Sh::S_COL0 + (it % Sh::SBUF) * NP + hcol, s);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sfree_bar[it & 1]);
+          if (lane == 0) mbar_arrive(&sfree_bar[it % Sh::SBUF]);
 
           if (first) {
 #pragma unroll
@@ -592,7 +608,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             for (int x = 0; x < HW; ++x) l_part[x] = first ? 0.f : l_part[x] * alpha[x];
             if (!first) {
               // O holds the sums up to tile it-1: wait for that PV, then rescale its columns
-              const bool okr = mbar_wait(&pvdone_bar[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag,
+              const bool okr = mbar_wait(&pvdone_bar[(it - 1) % Sh::PR], ((it - 1) / Sh::PR) & 1, abort_flag,
                                          p.wait_limit_ns);
               if (named_bar_or(bar_or, 128, !okr)) { ok = false; break; }
               tc_fence_after();
@@ -615,7 +631,8 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
           for (int x = 0; x < HW; x += 2)
             add_f32x2(l_part[x], l_part[x + 1], l_part[x], l_part[x + 1], pr[x], pr[x + 1]);
-          uint8_t* pbuf = pbufs + (it % Sh::PBUF) * Sh::P_BYTES;
+          uint8_t* pbuf = Sh::P_IN_STAGE ? stages + (it % STAGES) * Sh::STAGE_BYTES + Sh::NC * Sh::C_REG
+                                         : pbufs + (it % max(Sh::PBUF, 1)) * Sh::P_BYTES;
 #pragma unroll
           for (int c = 0; c < HW / 8; ++c) {
             uint4 w;
@@ -638,13 +655,13 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&pfull_bar[it & 1]);
+          if (lane == 0) mbar_arrive(&pfull_bar[it % Sh::PR]);
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 136 + min((int)it, 31));
           if (warp == 6 && lane == 0) MLRA_TRACE_POINT(1, 288 + min((int)it, 31));
 
           if (last) {
             // ---- segment epilogue: O / l and lse of this warpgroup's heads ----
-            const bool oke = mbar_wait(&pvdone_bar[it & 1], (it >> 1) & 1, abort_flag, p.wait_limit_ns);
+            const bool oke = mbar_wait(&pvdone_bar[it % Sh::PR], (it / Sh::PR) & 1, abort_flag, p.wait_limit_ns);
             if (named_bar_or(bar_or, 128, !oke || *abort_flag)) { ok = false; ++it; break; }
             tc_fence_after();
             float lt[HW];

@@ -27,13 +27,19 @@ namespace {
 // Compiled kernel set. A variant fixes (d_b, d_rope, heads per CTA, d_h) and the decode
 // kernel's shared-memory pipeline.
 // ---------------------------------------------------------------------------------------
-enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kNumVariants };
+enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kMlra4Sum = 4, kNumVariants };
 
 using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
-using DecMlra4 = DecodeShape<128, 64, 32, 4, 1, 2>;
+// P is written over each stage's RoPE columns, which leaves room for two query buffers (the
+// next segment's query loads while the current one is in use)
+using DecMlra4 = DecodeShape<128, 64, 32, 4, 2, 0>;
 using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
 // MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits
 using DecMla = DecodeShape<512, 64, 32, 1, 1, 2>;
+// MLRA-4 with summed blocks: all h heads attend to each block, so a CTA takes 64 heads (an
+// MMA of N = 64 costs the same issue time as N = 32); P lives in each stage's RoPE region so
+// that four 48 KB stages fit next to the 24 KB query
+using DecMlra4Sum = DecodeShape<128, 64, 64, 4, 1, 0>;
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 
@@ -41,7 +47,7 @@ struct VariantDims {
   int d_b, d_r, np, d_h;
 };
 constexpr VariantDims kDims[kNumVariants] = {
-    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 32, 128}};
+    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 32, 128}, {128, 64, 64, 128}};
 
 // Largest batch tile of the projection kernels: at d_b = 512 a 128-row tile of the merged
 // latent plus W^UV^T would need 256 KB of shared memory.
@@ -392,9 +398,17 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
         e = launch_decode<DecMlra4>(h, mc, mr, mqc, mqr, dp, s);
       rec(2);
       if (e == cudaSuccess)
-        e = latent      ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
-            : h->summed ? dispatch_uproj<512, 128, false, 4>(h, pp, batch, s)
-                        : dispatch_uproj<128, 128, false>(h, pp, batch, s);
+        e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<128, 128, false>(h, pp, batch, s);
+      break;
+    case kMlra4Sum:
+      e = dispatch_absorb<128, 128>(h, pp, batch, s);
+      rec(1);
+      if (e == cudaSuccess) e = launch_decode<DecMlra4Sum>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<512, 128, false, 4>(h, pp, batch, s);
       break;
     case kMlra2:
       e = dispatch_absorb<256, 128>(h, pp, batch, s);
@@ -480,13 +494,14 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   // heads per block: a group of h/k, or all h when every head attends to every block
   const int d_b = c.d_c / c.k, hb = summed ? c.h : c.h / c.k;
   int var = -1;
-  for (int v = 0; v < kNumVariants; ++v)
+  for (int v = 0; v < kMlra4Sum; ++v)  // the summed-only shapes are chosen below
     if (kDims[v].d_b == d_b && kDims[v].d_r == c.d_rope && kDims[v].d_h == c.d_h &&
         (hb <= kDims[v].np || hb % kDims[v].np == 0))
       var = v;
   if (var < 0) return MLRA_ERR_UNSUPPORTED;
   // summed blocks: the combine's GEMM runs over k*d_b, compiled for these two shapes
   if (summed && !((var == kMlra4 && c.k == 4) || (var == kTiny && c.k == 4))) return MLRA_ERR_UNSUPPORTED;
+  if (summed && var == kMlra4) var = kMlra4Sum;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLRA_ERR_CUDA;
@@ -525,8 +540,13 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
     case kMlra4:
       e = prep_decode<DecMlra4>();
       if (e == cudaSuccess) e = prep_proj_all<128, 128>();
-      if (e == cudaSuccess && summed) e = prep_proj_sum<512, 128, 4>();
       h->stages = DecMlra4::STAGES;
+      break;
+    case kMlra4Sum:
+      e = prep_decode<DecMlra4Sum>();
+      if (e == cudaSuccess) e = prep_proj_all<128, 128>();
+      if (e == cudaSuccess) e = prep_proj_sum<512, 128, 4>();
+      h->stages = DecMlra4Sum::STAGES;
       break;
     case kMlra2:
       e = prep_decode<DecMlra2>();

@@ -93,7 +93,8 @@ def test_summed_plan_is_bit_exact():
     inp = W.make_workload(w, device="cuda")
     hdl = _handle(w, inp)
     info = M.mlra_get_info(hdl)
-    assert info["ctas_per_group"] == 16 and info["groups"] == info["num_sms"] // 16
+    per = info["ctas_per_group"]
+    assert per == w.k * (w.h // info["heads_per_cta"]) and info["groups"] == info["num_sms"] // per
     rng = np.random.default_rng(8)
     for lens in (inp["seq_lens"].cpu().tolist(), [8192] * 32, list(rng.integers(0, 40000, 100))):
         sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
