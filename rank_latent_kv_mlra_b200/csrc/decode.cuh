@@ -88,8 +88,12 @@ struct DecodeShape {
   static constexpr int OFF_STAGES = 0;
   static constexpr int OFF_Q = OFF_STAGES + STAGES * STAGE_BYTES;
   static constexpr int OFF_P = OFF_Q + QBUF * Q_BYTES;
-  static constexpr int OFF_M = OFF_P + PBUF * P_BYTES;          // NP floats
-  static constexpr int OFF_RED = OFF_M + NP * 4;                // 4 x NP floats
+  // The running max per head is the same in every softmax thread. With 32 heads per warpgroup
+  // each warp keeps one copy in shared memory (read as broadcasts, written only when raised),
+  // which saves 32 registers per thread; with fewer heads it stays in registers.
+  static constexpr bool M_SMEM = HW >= 32;
+  static constexpr int OFF_M = OFF_P + PBUF * P_BYTES;          // running max: HW floats per softmax warp
+  static constexpr int OFF_RED = OFF_M + 4 * NWG * HW * 4;      // 4 x NP floats
   static constexpr int OFF_SEG = OFF_RED + 4 * NP * 4;          // MAX_SEGS segments
   static constexpr int OFF_BAR = round_up(OFF_SEG + MAX_SEGS * 16, 8);
   static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 2 * SBUF + 2 * PR + 2;
@@ -99,6 +103,7 @@ struct DecodeShape {
   static_assert(NP == 16 || NP == 32 || NP == 64, "heads per CTA");
   static_assert(QBUF == 1 || QBUF == 2, "query buffers");
   static_assert(SBUF >= 2 && TMEM_USED <= 512, "S buffers");
+  static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory of one sm_100 CTA");
   static_assert(PBUF == 0 || PBUF == 1 || PBUF == 2, "P buffers");
   static_assert(PBUF != 0 || P_BYTES <= NR * R_REG, "P must fit the RoPE region of a stage");
 };
@@ -536,9 +541,10 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       const int bar_or = 1 + 2 * g, bar_sync = 2 + 2 * g;
       const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
       float* red = red_sm + g * 4 * HW;
-      float m[HW];                        // running max per head (same in every thread)
-#pragma unroll
-      for (int x = 0; x < HW; ++x) m[x] = -INFINITY;
+      // running max per head (shared memory or registers, see DecodeShape::M_SMEM)
+      float m_reg[Sh::M_SMEM ? 1 : HW];
+      float* m_sm = reinterpret_cast<float*>(smem + Sh::OFF_M) + (warp - 2) * HW;
+      auto m = [&](int x) -> float& { return Sh::M_SMEM ? m_sm[x] : m_reg[x % (Sh::M_SMEM ? 1 : HW)]; };
       bool ok = true;
       for (int si = 0; si < nseg && ok; ++si) {
         const Segment sg = segs[si];
@@ -564,35 +570,47 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           if (lane == 0) mbar_arrive(&sfree_bar[it % Sh::SBUF]);
 
           if (first) {
+            // baseline 0 until the segment's first tile maximum is known, so that xs below
+            // holds the scores themselves
+            if constexpr (Sh::M_SMEM) {
+              __syncwarp();
+              for (int x = lane; x < HW; x += 32) m_sm[x] = 0.f;
+              __syncwarp();
+            } else {
 #pragma unroll
-            for (int x = 0; x < HW; ++x) m[x] = -INFINITY;
+              for (int x = 0; x < HW; ++x) m(x) = 0.f;
+            }
           }
-          // common case: scores relative to the running max, exp2 issued before the vote
+          // Common case: scores relative to the running max, exp2 issued before the vote. The
+          // raw scores are not kept: where the rare rescale path needs them it takes xs + m.
           float xs[HW];
 #pragma unroll
-          for (int x = 0; x < HW; x += 2) sub_f32x2(xs[x], xs[x + 1], s[x], s[x + 1], m[x], m[x + 1]);
+          for (int x = 0; x < HW; x += 2) sub_f32x2(xs[x], xs[x + 1], s[x], s[x + 1], m(x), m(x + 1));
           if (!tile_full && !valid) {
 #pragma unroll
             for (int x = 0; x < HW; ++x) xs[x] = -INFINITY;
           }
-          float dm[HW];
+          static_assert(HW % 4 == 0, "four max chains");
+          float d0 = xs[0], d1 = xs[1], d2 = xs[2], d3 = xs[3];
 #pragma unroll
-          for (int x = 0; x < HW; ++x) dm[x] = xs[x];
-#pragma unroll
-          for (int w2 = HW / 2; w2 >= 1; w2 >>= 1)
-#pragma unroll
-            for (int x = 0; x < w2; ++x) dm[x] = fmaxf(dm[x], dm[x + w2]);
+          for (int x = 4; x < HW; x += 4) {
+            d0 = fmaxf(d0, xs[x]);
+            d1 = fmaxf(d1, xs[x + 1]);
+            d2 = fmaxf(d2, xs[x + 2]);
+            d3 = fmaxf(d3, xs[x + 3]);
+          }
+          const float dmax = fmaxf(fmaxf(d0, d1), fmaxf(d2, d3));
           float pr[HW];
 #pragma unroll
           for (int x = 0; x < HW; ++x) pr[x] = fast_exp2(xs[x]);
 
-          const bool need = named_bar_or(bar_or, 128, !okl || first || dm[0] > kRescaleSlack);
+          const bool need = named_bar_or(bar_or, 128, !okl || first || dmax > kRescaleSlack);
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 256 + min((int)it, 31));
           if (need) {
             if (named_bar_or(bar_or, 128, !okl || *abort_flag)) { ok = false; break; }
             float tmax[HW];
 #pragma unroll
-            for (int x = 0; x < HW; ++x) tmax[x] = valid ? s[x] : -INFINITY;
+            for (int x = 0; x < HW; ++x) tmax[x] = valid ? xs[x] + m(x) : -INFINITY;
             warp_reduce_scatter<HW, true>(tmax, lane);
             store_scattered<HW>(tmax, red + q4 * HW, lane);
             named_bar_sync(bar_sync, 128);
@@ -600,9 +618,21 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
             for (int x = 0; x < HW; ++x) {
               const float tm = fmaxf(fmaxf(red[x], red[HW + x]), fmaxf(red[2 * HW + x], red[3 * HW + x]));
-              const float mn = fmaxf(m[x], tm);
-              alpha[x] = first ? 0.f : fast_exp2(m[x] - mn);
-              m[x] = mn;
+              const float mo = m(x);
+              const float mn = first ? tm : fmaxf(mo, tm);
+              alpha[x] = first ? 0.f : fast_exp2(mo - mn);
+              pr[x] = valid ? fast_exp2((xs[x] + mo) - mn) : 0.f;
+              if constexpr (!Sh::M_SMEM) m(x) = mn;
+            }
+            if constexpr (Sh::M_SMEM) {
+              // raise the warp's copy once every lane has read the old values (red stays intact
+              // until the barrier below)
+              __syncwarp();
+              for (int x = lane; x < HW; x += 32) {
+                const float tm = fmaxf(fmaxf(red[x], red[HW + x]), fmaxf(red[2 * HW + x], red[3 * HW + x]));
+                m_sm[x] = first ? tm : fmaxf(m_sm[x], tm);
+              }
+              __syncwarp();
             }
 #pragma unroll
             for (int x = 0; x < HW; ++x) l_part[x] = first ? 0.f : l_part[x] * alpha[x];
@@ -625,8 +655,6 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
               tmem_st_wait();
             }
             named_bar_sync(bar_sync, 128);  // everyone has read red
-#pragma unroll
-            for (int x = 0; x < HW; ++x) pr[x] = valid ? fast_exp2(s[x] - m[x]) : 0.f;
           }
 #pragma unroll
           for (int x = 0; x < HW; x += 2)
@@ -676,7 +704,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
               const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
               inv[x] = 1.f / l;
               if (sw == 0 && x % 32 == lane && hcol + x < nheads)
-                p.lse_part[(size_t)slot * p.h + head0 + hcol + x] = m[x] + __log2f(l);
+                p.lse_part[(size_t)slot * p.h + head0 + hcol + x] = m(x) + __log2f(l);
             }
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {

@@ -34,8 +34,10 @@ using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 // next segment's query loads while the current one is in use)
 using DecMlra4 = DecodeShape<128, 64, 32, 4, 2, 0>;
 using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
-// MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits
-using DecMla = DecodeShape<512, 64, 32, 1, 1, 2>;
+// MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits; 64
+// heads per CTA (2 CTAs per group) halve the MMA work per cached byte against 32, and P goes
+// into the stage so the 72 KB query fits beside it
+using DecMla = DecodeShape<512, 64, 64, 1, 1, 0>;
 // MLRA-4 with summed blocks: all h heads attend to each block, so a CTA takes 64 heads (an
 // MMA of N = 64 costs the same issue time as N = 32); P lives in each stage's RoPE region so
 // that four 48 KB stages fit next to the 24 KB query
@@ -47,7 +49,7 @@ struct VariantDims {
   int d_b, d_r, np, d_h;
 };
 constexpr VariantDims kDims[kNumVariants] = {
-    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 32, 128}, {128, 64, 64, 128}};
+    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 64, 128}, {128, 64, 64, 128}};
 
 // Largest batch tile of the projection kernels: at d_b = 512 a 128-row tile of the merged
 // latent plus W^UV^T would need 256 KB of shared memory.
