@@ -76,6 +76,12 @@ struct DecodeShape {
   static constexpr int P_ROWB = NP * 2;
   static constexpr int P_BYTES = round_up(kTile * P_ROWB, 1024);
   static constexpr int NMT = DB >= 128 ? DB / 128 : 1;  // PV M tiles
+  // A stage is loaded and freed in NG groups, one per PV M tile (128 latent features); the RoPE
+  // columns, and P written over them, belong to the last group. A group is reloaded as soon as
+  // the PV MMAs of its M tile have read it, so with several M tiles (d_b = 256, 512) the next
+  // tile's first columns stream in while this tile's PV is still running.
+  static constexpr int NG = NMT;
+  static constexpr int RPG = (DB / (DB < 64 ? DB : 64)) / NMT;  // block regions per group
   static constexpr uint32_t PV_LBO = DB >= 128 ? C_REG : 0;  // next 64-feature chunk
   static constexpr int SBUF = SBUF_;                // S buffers of NP columns in TMEM
   static constexpr int S_COL0 = 0;
@@ -96,7 +102,9 @@ struct DecodeShape {
   static constexpr int OFF_RED = OFF_M + 4 * NWG * HW * 4;      // 4 x NP floats
   static constexpr int OFF_SEG = OFF_RED + 4 * NP * 4;          // MAX_SEGS segments
   static constexpr int OFF_BAR = round_up(OFF_SEG + MAX_SEGS * 16, 8);
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * QBUF + 2 * SBUF + 2 * PR + 2;
+  static constexpr int NUM_BARS = 2 * STAGES * NG + 2 * QBUF + 2 * SBUF + 2 * PR + 2;
+  // bytes one page brings into group g
+  static constexpr int group_tx(int g) { return RPG * kPage * C_ROWB + (g == NG - 1 ? NR * kPage * R_ROWB : 0); }
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem slot, flags, scratch
   static constexpr int SMEM_BYTES = OFF_MISC + 64 * 4 + 1024;  // + alignment slack
   static_assert(DB % CW == 0 && DR % RW == 0, "region split");
@@ -104,6 +112,7 @@ struct DecodeShape {
   static_assert(QBUF == 1 || QBUF == 2, "query buffers");
   static_assert(SBUF >= 2 && TMEM_USED <= 512, "S buffers");
   static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory of one sm_100 CTA");
+  static_assert(NG * RPG == NC && STAGES * NG <= 32, "column groups");
   static_assert(PBUF == 0 || PBUF == 1 || PBUF == 2, "P buffers");
   static_assert(PBUF != 0 || P_BYTES <= NR * R_REG, "P must fit the RoPE region of a stage");
 };
@@ -212,9 +221,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   float* red_sm = reinterpret_cast<float*>(smem + Sh::OFF_RED);
   Segment* segs = reinterpret_cast<Segment*>(smem + Sh::OFF_SEG);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::OFF_BAR);
-  uint64_t* full_bar = bars;
-  uint64_t* empty_bar = bars + STAGES;
-  uint64_t* qfull_bar = bars + 2 * STAGES;
+  uint64_t* full_bar = bars;                         // [stage][group]
+  uint64_t* empty_bar = bars + STAGES * Sh::NG;       // [stage][group]
+  uint64_t* qfull_bar = bars + 2 * STAGES * Sh::NG;
   uint64_t* qempty_bar = qfull_bar + Sh::QBUF;
   uint64_t* sfull_bar = qempty_bar + Sh::QBUF;
   uint64_t* sfree_bar = sfull_bar + Sh::SBUF;
@@ -239,7 +248,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < STAGES * Sh::NG; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -296,8 +305,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   // pipeline counters persist across segment-list refills
   uint32_t it = 0;      // tiles consumed/produced so far by this role
   uint32_t segc = 0;    // segments so far
-  // producer: last issued phase per stage, for the drain at the end
-  uint32_t issued_mask = 0;
+  // producer: which (stage, group) barriers have a load issued and the parity of the last
+  // issued phase of each, for the drain at the end
+  uint32_t issued_mask = 0, issued_phase = 0;
   // softmax-role partial sums (the warpgroup's heads)
   float l_part[Sh::HW];
 #pragma unroll
@@ -404,20 +414,26 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             if (id0 < 0 || id0 >= p.num_pages) { set_status(p.status, kErrPageOob); id0 = 0; }
             if (npg == 2 && (id1 < 0 || id1 >= p.num_pages)) { set_status(p.status, kErrPageOob); id1 = 0; }
             const int st = it % STAGES;
-            ok = mbar_wait(&empty_bar[st], ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_limit_ns);
-            if (ok && !(p.inject_stall && it == 0)) {
-              MLRA_TRACE_POINT(1, 8 + min((int)it, 31));
-              uint8_t* dst = stages + st * Sh::STAGE_BYTES;
-              mbar_arrive_expect_tx(&full_bar[st], npg * Sh::PAGE_TX);
-              issued_mask |= 1u << st;
-              for (int pg = 0; pg < npg; ++pg) {
-                const int y = (pg ? id1 : id0) * kPage;
-                for (int r = 0; r < Sh::NC; ++r)
-                  tma_load_2d(dst + r * Sh::C_REG + pg * kPage * Sh::C_ROWB, &map_c, &full_bar[st],
-                              blk * Sh::DB + r * Sh::CW, y, pol_stream);
-                for (int r = 0; r < Sh::NR; ++r)
-                  tma_load_2d(dst + Sh::NC * Sh::C_REG + r * Sh::R_REG + pg * kPage * Sh::R_ROWB,
-                              &map_r, &full_bar[st], p.d_c + r * Sh::RW, y, pol_keep);
+            const uint32_t ph = (it / STAGES) & 1;
+            uint8_t* dst = stages + st * Sh::STAGE_BYTES;
+            for (int g = 0; g < Sh::NG && ok; ++g) {
+              const int gi = st * Sh::NG + g;
+              ok = mbar_wait(&empty_bar[gi], ph ^ 1, abort_flag, p.wait_limit_ns);
+              if (ok && !(p.inject_stall && it == 0)) {
+                if (g == 0) MLRA_TRACE_POINT(1, 8 + min((int)it, 31));
+                mbar_arrive_expect_tx(&full_bar[gi], npg * Sh::group_tx(g));
+                issued_mask |= 1u << gi;
+                issued_phase = (issued_phase & ~(1u << gi)) | (ph << gi);
+                for (int pg = 0; pg < npg; ++pg) {
+                  const int y = (pg ? id1 : id0) * kPage;
+                  for (int r = g * Sh::RPG; r < (g + 1) * Sh::RPG; ++r)
+                    tma_load_2d(dst + r * Sh::C_REG + pg * kPage * Sh::C_ROWB, &map_c, &full_bar[gi],
+                                blk * Sh::DB + r * Sh::CW, y, pol_stream);
+                  if (g == Sh::NG - 1)
+                    for (int r = 0; r < Sh::NR; ++r)
+                      tma_load_2d(dst + Sh::NC * Sh::C_REG + r * Sh::R_REG + pg * kPage * Sh::R_ROWB,
+                                  &map_r, &full_bar[gi], p.d_c + r * Sh::RW, y, pol_keep);
+                }
               }
             }
           }
@@ -439,41 +455,48 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           const int qb = sc % Sh::QBUF;
           ok = mbar_wait(&qfull_bar[qb], (sc / Sh::QBUF) & 1, abort_flag, p.wait_limit_ns);
           for (int t = sg.tile_begin; t < sg.tile_end && ok; ++t, ++ci) {
-            ok = mbar_wait(&full_bar[ci % STAGES], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
-            MLRA_TRACE_POINT(1, 400 + min((int)ci, 31));
-            if (ok && ci >= Sh::SBUF)
+            if (ci >= Sh::SBUF)
               ok = mbar_wait(&sfree_bar[ci % Sh::SBUF], ((ci / Sh::SBUF) - 1) & 1, abort_flag, p.wait_limit_ns);
             MLRA_TRACE_POINT(1, 432 + min((int)ci, 31));
-            if (!ok) break;
-            tc_fence_after();
-            MLRA_TRACE_POINT(1, 40 + min((int)ci, 31));
             const uint32_t st_addr = smem_u32(stages + (ci % STAGES) * Sh::STAGE_BYTES);
             const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
             const uint32_t d = tbase + Sh::S_COL0 + (ci % Sh::SBUF) * NP;
             uint32_t acc = 0;
+            // each column group's MMAs go out as soon as that group has landed
 #pragma unroll
-            for (int r = 0; r < Sh::NC; ++r) {
+            for (int g = 0; g < Sh::NG; ++g) {
+              if (ok) ok = mbar_wait(&full_bar[(ci % STAGES) * Sh::NG + g], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
+              if (!ok) break;
+              if (g == 0) MLRA_TRACE_POINT(1, 400 + min((int)ci, 31));
+              tc_fence_after();
 #pragma unroll
-              for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
-                const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                             swizzle_code(Sh::C_ROWB));
-                const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
-                                             swizzle_code(Sh::C_ROWB));
-                umma_bf16(d, a, b, idesc_qk, acc);
-                acc = 1;
+              for (int r = g * Sh::RPG; r < (g + 1) * Sh::RPG; ++r) {
+#pragma unroll
+                for (int ks = 0; ks < Sh::C_ROWB / 32; ++ks) {
+                  const uint64_t a = smem_desc(st_addr + r * Sh::C_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                               swizzle_code(Sh::C_ROWB));
+                  const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
+                                               swizzle_code(Sh::C_ROWB));
+                  umma_bf16(d, a, b, idesc_qk, acc);
+                  acc = 1;
+                }
+              }
+              if (g == Sh::NG - 1) {
+#pragma unroll
+                for (int r = 0; r < Sh::NR; ++r) {
+#pragma unroll
+                  for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
+                    const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
+                                                 8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                    const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
+                                                 8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
+                    umma_bf16(d, a, b, idesc_qk, 1);
+                  }
+                }
               }
             }
-#pragma unroll
-            for (int r = 0; r < Sh::NR; ++r) {
-#pragma unroll
-              for (int ks = 0; ks < Sh::R_ROWB / 32; ++ks) {
-                const uint64_t a = smem_desc(st_addr + Sh::NC * Sh::C_REG + r * Sh::R_REG + ks * 32, 16,
-                                             8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
-                                             8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                umma_bf16(d, a, b, idesc_qk, 1);
-              }
-            }
+            MLRA_TRACE_POINT(1, 40 + min((int)ci, 31));
+            if (!ok) break;
             umma_commit(&sfull_bar[ci % Sh::SBUF]);
             if (t == sg.tile_end - 1) umma_commit(&qempty_bar[qb]);
           }
@@ -516,8 +539,10 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                                              swizzle_code(Sh::P_ROWB));
                 umma_bf16(tbase + Sh::O_COL + mt * NP, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
               }
+              // this M tile's columns are read: its group may be reloaded (the last group also
+              // holds the RoPE columns and P, read by every M tile)
+              umma_commit(&empty_bar[(pi % STAGES) * Sh::NG + mt]);
             }
-            umma_commit(&empty_bar[pi % STAGES]);
             umma_commit(&pvdone_bar[pi % Sh::PR]);
           }
         }
@@ -733,12 +758,10 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 200);
   // ---- teardown: nothing may be in flight when shared memory and TMEM are released ----
   if (warp == 0 && lane == 0) {
-    // wait for every stage's last issued load (completed loads return at once)
-    for (int s = 0; s < STAGES; ++s) {
-      if (!(issued_mask & (1u << s))) continue;
-      // the last tile that used stage s
-      const uint32_t last_it = it == 0 ? 0 : (it - 1) - ((it - 1 + STAGES - s) % STAGES);
-      mbar_wait_drain(&full_bar[s], (last_it / STAGES) & 1, p.wait_limit_ns);
+    // wait for the last issued load of every (stage, group) (completed loads return at once)
+    for (int gi = 0; gi < STAGES * Sh::NG; ++gi) {
+      if (!(issued_mask & (1u << gi))) continue;
+      mbar_wait_drain(&full_bar[gi], (issued_phase >> gi) & 1, p.wait_limit_ns);
     }
   }
   if (warp == 1 || warp == Sh::PV_WARP) {
