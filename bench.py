@@ -407,7 +407,7 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": step_ms_max, "us_per_step": step_ms_max * 1e3,
         "pct_of_hbm_peak": 100.0 * value / world / peak,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; inputs larger than L2: the 302 MB cache stream evicts the 126 MB L2 each step)",
+        "data": f"synthetic (seeded; inputs larger than L2: the {nbytes / 1e6:.0f} MB cache stream evicts the 126 MB L2 each step)",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
                    "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
                    "reading": "summed" if w.summed else "partitioned",

@@ -72,7 +72,6 @@ struct DecodeShape {
   static constexpr int QC_REG = round_up(NP * C_ROWB, 1024);
   static constexpr int QR_REG = round_up(NP * R_ROWB, 1024);
   static constexpr int Q_BYTES = NC * QC_REG + NR * QR_REG;
-  static constexpr int Q_TX = NP * (DB + DR) * 2;
   static constexpr int P_ROWB = NP * 2;
   static constexpr int P_BYTES = round_up(kTile * P_ROWB, 1024);
   static constexpr int NMT = DB >= 128 ? DB / 128 : 1;  // PV M tiles
@@ -129,6 +128,7 @@ struct DecodeParams {
   int heads_block;  // h / k
   int h;            // total heads
   int d_c;          // column of k^R in a cache row
+  int q_rows;       // query rows a CTA loads: min(h/k, NP); rows past them stay zero
   float* o_part;    // [slots][h][DB] fp32, normalised partial latent outputs
   float* lse_part;  // [slots][h] fp32, log2-domain log-sum-exp
   int* status;
@@ -280,6 +280,21 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
     tmem_alloc(tmem_slot, Sh::TMEM_COLS);
     tmem_relinquish();
   }
+  if (p.q_rows < NP) {
+    // Head chunks narrower than the MMA's N (h/k < NP): the query loads bring q_rows rows, and
+    // the rows past them, which no load ever writes, are zero for the whole launch. A swizzled
+    // row keeps its bytes within its own row span, so whole rows are cleared.
+    for (int qb = 0; qb < Sh::QBUF; ++qb) {
+      uint8_t* qdst = qbufs + qb * Sh::Q_BYTES;
+      for (int r = 0; r < Sh::NC; ++r)
+        for (int i = p.q_rows * Sh::C_ROWB + threadIdx.x * 16; i < NP * Sh::C_ROWB; i += Sh::THREADS * 16)
+          *reinterpret_cast<uint4*>(qdst + r * Sh::QC_REG + i) = make_uint4(0, 0, 0, 0);
+      for (int r = 0; r < Sh::NR; ++r)
+        for (int i = p.q_rows * Sh::R_ROWB + threadIdx.x * 16; i < NP * Sh::R_ROWB; i += Sh::THREADS * 16)
+          *reinterpret_cast<uint4*>(qdst + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + i) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -372,7 +387,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           ok = mbar_wait(&qempty_bar[qb], ((segc / Sh::QBUF) & 1) ^ 1, abort_flag, p.wait_limit_ns);
           if (ok) {
             uint8_t* qdst = qbufs + qb * Sh::Q_BYTES;
-            mbar_arrive_expect_tx(&qfull_bar[qb], Sh::Q_TX);
+            mbar_arrive_expect_tx(&qfull_bar[qb], p.q_rows * (Sh::DB + Sh::DR) * 2);
             const int qrow = (sg.b * p.nsub + sub) * NP;
             for (int r = 0; r < Sh::NC; ++r)
               tma_load_2d(qdst + r * Sh::QC_REG, &map_qc, &qfull_bar[qb], r * Sh::CW, qrow, pol_keep);

@@ -321,10 +321,12 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   const int cw = h->d_b < 64 ? h->d_b : 64, rw = h->d_r < 64 ? h->d_r : 64;
   CUtensorMap mc, mr, mqc, mqr;
   const uint64_t qrows = (uint64_t)batch * h->nsub * h->np;
+  // a head chunk narrower than the MMA's N loads only its real rows
+  const uint32_t q_rows = h->heads_block < h->np ? h->heads_block : h->np;
   if (!make_map(&mc, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, cw) ||
       !make_map(&mr, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, rw) ||
-      !make_map(&mqc, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, h->np, cw) ||
-      !make_map(&mqr, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, h->np, rw))
+      !make_map(&mqc, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, q_rows, cw) ||
+      !make_map(&mqr, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, q_rows, rw))
     return MLRA_ERR_CUDA;
 
   ProjParams pp = {};
@@ -366,6 +368,7 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   dp.heads_block = h->heads_block;
   dp.h = h->vh;
   dp.d_c = h->cfg.d_c;
+  dp.q_rows = (int)q_rows;
   dp.o_part = w.o_part;
   dp.lse_part = w.lse_part;
   dp.status = w.status;

@@ -227,17 +227,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
   }
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 11);
-  // rows of a head chunk that no head fills (h/k below the MMA width) are zero
-  if (hb == p.heads_block - 1 && prow == hb % p.np) {
-    const int pad = p.np - 1 - prow;
-    for (int idx = threadIdx.x; idx < NT * pad * qw; idx += kProjThreads) {
-      const int bl = idx / (pad * qw), rest = idx % (pad * qw);
-      const int b = n0 + bl;
-      if (b >= p.batch) continue;
-      p.q_pack[(((size_t)b * p.nsub + sub) * p.np + prow + 1 + rest / qw) * qw + rest % qw] =
-          __float2bfloat16_rn(0.f);
-    }
-  }
+  // rows of a head chunk that no head fills (h/k below the MMA width) are never read: the
+  // decode kernel loads only the real rows and keeps the rest zero in shared memory
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 12);
   fence_proxy_async_smem();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 13);

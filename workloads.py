@@ -75,6 +75,14 @@ WORKLOADS = {
         # the summed-blocks reading of MLRA-4 on the headline's shapes
         Workload("mlra4sum_h128_b32_n8192", k=4, h=128, d_h=128, d_c=512, d_r=64, batch=32,
                  seq_len=8192, seed=5, summed=True),
+        # One rank's share under 4-way tensor parallelism of the headline's model (h = 128,
+        # d_c = 512, d_r = 64): an MLRA-4 rank holds one block plus the RoPE key and its 32
+        # heads; an MLA rank holds the whole latent and 32 heads. Batch 64 keeps either cache
+        # larger than L2.
+        Workload("tp4rank_mlra4_h32_b64_n8192", k=1, h=32, d_h=128, d_c=128, d_r=64, batch=64,
+                 seq_len=8192, seed=6),
+        Workload("tp4rank_mla_h32_b64_n8192", k=1, h=32, d_h=128, d_c=512, d_r=64, batch=64,
+                 seq_len=8192, seed=6),
     ]
 }
 
