@@ -222,7 +222,7 @@ cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cu
       return cudaErrorInvalidValue;
   }
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->vh, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, false,
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->vh, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, true,
                                     &attr);
   return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, mqc, mqr, pp);
 }

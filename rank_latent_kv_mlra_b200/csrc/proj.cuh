@@ -126,7 +126,6 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int prow = hb % p.np;
 
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 0);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.status) *p.status = 0;
   // a bf16 query comes in by TMA with the weight: [batch tile][q^C columns] straight into the
   // MMA's swizzled B layout, [batch tile][q^R] into a staging tile (rows past the batch read 0)
   const bool tma_q = !p.q_f32;
@@ -135,12 +134,17 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     mbar_init(&bars[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // issue the loads first: nothing below depends on them until the MMA
+    // issue the loads first: nothing below depends on them until the MMA. The weight does not
+    // depend on the previous kernel in the stream, so it streams in while that kernel finishes
+    // (programmatic dependent launch); the query, the status word and the packed-query output
+    // wait for it.
     const uint64_t pol = l2_policy_evict_first();
     mbar_arrive_expect_tx(&bars[0], Sh::A1_TX + (tma_q ? NT * (DH + p.d_r) * 2 : 0));
     for (int kr = 0; kr < Sh::NKR; ++kr)
       for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
         tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW, head * DB + r0, pol);
+    grid_dependency_wait();
+    if (blockIdx.x == 0 && blockIdx.y == 0 && p.status) *p.status = 0;
     if (tma_q) {
       const int qh = head % p.q_heads;
       for (int kr = 0; kr < Sh::NKR; ++kr)
@@ -155,6 +159,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dependency_wait();  // (returns at once: thread 0 has waited for the previous kernel)
   const uint32_t tbase = *tmem_slot;
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 1);
   // let the decode kernel's CTAs start (on SMs this grid leaves free) and run their set-up and
@@ -421,6 +426,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 1);
 
   grid_dependency_wait();  // the partials come from the decode kernel
+  // the next kernel in the stream (the next step's absorb) may start its set-up and weight
+  // loads now; it waits for this grid before touching anything this grid reads or writes
+  grid_launch_dependents();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 2);
 
   // merge the split partials of each (sequence, head) and stage o~ as bf16 (K-major).
