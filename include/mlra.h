@@ -110,7 +110,10 @@ int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes);
  *   workspace  device, >= mlra_workspace_size(batch) bytes, 256-byte aligned. Its first
  *              4 bytes become this call's status word.
  * Launches three kernels on `stream`: query absorption, split-KV latent attention, and
- * log-sum-exp combine fused with the W^UV up-projection. */
+ * log-sum-exp combine fused with the W^UV up-projection. All three use programmatic
+ * dependent launch: the first may begin loading W^UK and setting up while the kernel before
+ * it on `stream` finishes, and reads q (and writes the workspace) only after that kernel has
+ * completed; stream order is otherwise unchanged. */
 int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
                 int num_pages, const int32_t* page_table, int pt_stride,
                 const int32_t* seq_lens, int batch, void* out, mlra_dtype out_dtype,
