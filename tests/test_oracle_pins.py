@@ -245,6 +245,29 @@ def test_block_independence():
         assert not changed[mask].any()
 
 
+@pytest.mark.parametrize("k", [2, 4])
+def test_tensor_parallel_shards_reproduce_the_layer(k):
+    """k-way tensor parallelism (alanhou.org summary, Core Mechanism: each device loads only its
+    latent head's cache, computes its subset of heads, and the results are combined): rank j
+    runs plain latent attention (k = 1) over [c_j | k^R] with head group j's query and
+    matrices; concatenating the ranks' heads gives the MLRA-k layer's output and lse."""
+    rng = np.random.default_rng(20 + k)
+    case = _rand_case(rng, k=k, d_b=48 // k * 2)
+    full = _run(case, scale=0.4)
+    h, d_b, d_c = case["h"], case["d_c"] // k, case["d_c"]
+    hb = h // k
+    outs, lses = [], []
+    for j in range(k):
+        shard = np.concatenate([case["pool"][..., j * d_b:(j + 1) * d_b], case["pool"][..., d_c:]], axis=-1)
+        g = slice(j * hb, (j + 1) * hb)
+        r = O.decode(case["q"][:, g], case["w_uk"][g], case["w_uv"][g], shard, case["page_table"],
+                     case["seq_lens"], 1, case["d_r"], scale=0.4)
+        outs.append(r["out"])
+        lses.append(r["lse"])
+    np.testing.assert_allclose(np.concatenate(outs, axis=1), full["out"], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(np.concatenate(lses, axis=1), full["lse"], rtol=1e-13, atol=1e-14)
+
+
 def test_page_placement_and_key_order_invariance():
     rng = np.random.default_rng(7)
     case = _rand_case(rng, permute=False)
