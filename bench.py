@@ -435,6 +435,73 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def producer_bytes(w, batch, d_model):
+    """Algorithmic bytes of the new-row step: bf16 weights [d_c + d_r][d_model] and hidden
+    states read once, bf16 rows written, one position and one page-table entry per token."""
+    d_out = w.d_c + w.d_r
+    return 2 * d_out * d_model + 2 * batch * d_model + 2 * batch * d_out + 8 * batch
+
+
+def run_producer(args, world, rank, local):
+    """Times the step before decoding (each sequence's new cache row: down-projection, RoPE
+    key, page slot) on the workload's batch with d_model = workloads.PRODUCER_D_MODEL. Its
+    inputs (about 6 MB) fit in L2, so L2 is flushed (a 256 MB write) before every timed step
+    and each step is timed alone with CUDA events."""
+    import rank_latent_kv_mlra_b200 as M
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_workload(w, device=dev)
+    pr = W.make_producer_inputs(w, inp)
+    hdl = M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed)
+    d_model = pr["d_model"]
+    ws = torch.empty(M.mlra_project_workspace_size(hdl, w.batch, d_model), dtype=torch.uint8, device=dev)
+    call = lambda: M.mlra_project_append(hdl, pr["x"], pr["w_down"], pr["positions"], inp["pool"],
+                                         inp["page_table"], workspace=ws)
+    call()
+    torch.cuda.synchronize()
+    if M.mlra_get_status(ws) != 0:
+        raise RuntimeError(f"producer status {M.mlra_get_status(ws)}")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    stream = torch.cuda.current_stream(dev)
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    ms = max_over_ranks(ms, world, dev)
+    if rank != 0:
+        return
+    nbytes = producer_bytes(w, w.batch, d_model)
+    peak, peak_kind = measured_hbm_peak()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "new cache rows (x W^DKV | RoPE(x W^KR), stored in their page slots): achieved HBM GB/s",
+        "value": world * gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; L2 flushed by a 256 MB write before each step)",
+        "config": {"workload": w.name, "batch": w.batch, "d_model": d_model, "d_c": w.d_c, "d_r": w.d_r,
+                   "l2": "flushed before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "bytes_per_step": nbytes,
+                     "kernel": "mlra_down_proj_kernel + mlra_rope_append_kernel", "traffic": None},
+        "gpu_launches": 2 * args.steps, "clocks": clk,
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -444,6 +511,8 @@ def main():
     ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
     ap.add_argument("--cpu-pairs", type=int, default=15000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--producer", action="store_true",
+                    help="time the step before decoding (the new cache rows) instead of the decode step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -451,6 +520,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.producer:
+            run_producer(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

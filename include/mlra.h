@@ -173,6 +173,40 @@ int mlra_append_cache(mlra_handle h, void* pool, int num_pages, const int32_t* p
                       const void* c_new, const void* kr_new, mlra_dtype in_dtype,
                       int n_tokens, int32_t* status, void* stream);
 
+/* Bytes of device workspace mlra_project_append needs (host output). d_model must be a
+ * multiple of 128. */
+int mlra_project_workspace_size(mlra_handle h, int batch, int d_model, size_t* bytes);
+
+/* The step before decoding: computes each sequence's new cache row and stores it.
+ * For token b with hidden state x[b] at position positions[b] (0-based index in its sequence):
+ *   c   = x[b] W^DKV       (d_c latent features, all k blocks; the down-projection that the
+ *                           "Multi-Head Low-Rank Attention: Making Compressed Attention Actually
+ *                           Parallelizable" page's Core Mechanism and the lesty.tech MLA
+ *                           article's section 4 describe)
+ *   k^R = RoPE(x[b] W^KR)  (d_rope features; feature pair (2i, 2i+1) rotated by the angle
+ *                           pos * rope_base^(-2i/d_rope), RoFormer's rotation, which the pages
+ *                           cite but do not spell out)
+ * and writes the bf16 (round to nearest even) row [c | k^R] into slot pos % page_size of page
+ * page_table[b*pt_stride + pos/page_size].
+ *   x          device bf16 [batch][d_model], 16-byte aligned; d_model a multiple of 128.
+ *   w_down     device bf16 [d_c + d_rope][d_model], 16-byte aligned: row r holds the weights
+ *              of output feature r (the d_c latent features, then the d_rope RoPE-key
+ *              features), i.e. W^DKV and W^KR transposed and stacked. Borrowed for the call.
+ *   rope_base  RoPE base; <= 1 selects 10000.
+ *   positions  device int32 [batch]; 0 <= pos < pt_stride * page_size, else the row is not
+ *              written and the status word reads MLRA_ERR_SEQ_LEN.
+ *   pool, num_pages, page_table, pt_stride: as in mlra_decode; a page id outside
+ *              [0, num_pages) leaves the row unwritten and reports MLRA_ERR_PAGE_OOB.
+ *   workspace  device, >= mlra_project_workspace_size bytes, 256-byte aligned; its first 4
+ *              bytes become this call's status word (read it with mlra_get_status).
+ * Launches two kernels on `stream` (a split-d_model tcgen05 GEMM into fp32 partials, then the
+ * sum / rotation / store), both under programmatic dependent launch: the first loads W^DKV
+ * while the previous kernel on `stream` finishes and reads x only after it has completed.
+ * Rows of one call must go to distinct slots. */
+int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w_down, float rope_base,
+                        const int32_t* positions, void* pool, int num_pages, const int32_t* page_table,
+                        int pt_stride, int batch, void* workspace, size_t ws_bytes, void* stream);
+
 /* Runs the device split planner on seq_lens and writes the segments it would process:
  * segments device int32 [max_segments][5] rows (b, group, tile_begin, tile_end, slot),
  * count device int32. A group is a set of CTAs that shares one run of 128-token tiles;

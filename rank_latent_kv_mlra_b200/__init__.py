@@ -35,7 +35,7 @@ STATUS = {
 EXPORTED = [
     "mlra_create", "mlra_destroy", "mlra_workspace_size", "mlra_decode", "mlra_decode_latent",
     "mlra_append_cache", "mlra_plan", "mlra_get_info", "mlra_get_status", "mlra_status_string",
-    "mlra_decode_profiled", "mlra_decode_noalloc",
+    "mlra_decode_profiled", "mlra_decode_noalloc", "mlra_project_workspace_size", "mlra_project_append",
 ]
 
 
@@ -80,6 +80,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mlra_decode_latent.argtypes = [P, P, I, P, I, P, I, P, I, P, P, P, S, P]
     lib.mlra_decode_profiled.argtypes = [P, P, I, P, I, P, I, P, I, P, I, P, P, S, P, P]
     lib.mlra_append_cache.argtypes = [P, P, I, P, I, I, P, P, P, P, I, I, P, P]
+    lib.mlra_project_workspace_size.argtypes = [P, I, I, ctypes.POINTER(S)]
+    lib.mlra_project_append.argtypes = [P, P, I, P, ctypes.c_float, P, P, I, P, I, I, P, S, P]
     lib.mlra_plan.argtypes = [P, P, I, I, P, I, P, P]
     lib.mlra_get_info.argtypes = [P, ctypes.POINTER(mlra_info)]
     lib.mlra_get_status.argtypes = [P, ctypes.POINTER(I)]
@@ -279,6 +281,40 @@ def mlra_append_cache(handle: Handle, pool, page_table, seq_ids, positions, c_ne
         handle.ptr, _ptr(pool), pool.shape[0], _ptr(page_table), page_table.shape[1],
         page_table.shape[0], _ptr(seq_ids), _ptr(positions), _ptr(c_new), _ptr(kr_new),
         _dtype(c_new), seq_ids.numel(), _ptr(status), _stream(stream)), "mlra_append_cache")
+
+
+def mlra_project_workspace_size(handle: Handle, batch: int, d_model: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().mlra_project_workspace_size(handle.ptr, batch, d_model, ctypes.byref(n)),
+           "mlra_project_workspace_size")
+    return n.value
+
+
+def mlra_project_append(handle: Handle, x, w_down, positions, pool, page_table, rope_base=10000.0,
+                        workspace=None, stream=None):
+    """The new token's cache row [x W^DKV | RoPE(x W^KR)] of each sequence, stored at its
+    position. x bf16 [batch][d_model]; w_down bf16 [d_c + d_rope][d_model]; positions int32
+    [batch]. Returns the workspace, whose first int32 is the call's status word."""
+    _require(x, "x", torch.bfloat16)
+    _require(w_down, "w_down", torch.bfloat16)
+    _require(positions, "positions", torch.int32)
+    _require(pool, "pool", torch.bfloat16)
+    _require(page_table, "page_table", torch.int32)
+    cfg = handle.cfg
+    B, d_model = x.shape
+    if tuple(w_down.shape) != (cfg.d_c + cfg.d_rope, d_model):
+        raise ValueError("w_down must be [d_c + d_rope][d_model]")
+    if positions.shape != (B,) or page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("positions must be [batch], page_table [batch][pt_stride]")
+    if workspace is None:
+        workspace = torch.empty(mlra_project_workspace_size(handle, B, d_model), dtype=torch.uint8,
+                                device=x.device)
+    _require(workspace, "workspace")
+    _check(load_library().mlra_project_append(
+        handle.ptr, _ptr(x), d_model, _ptr(w_down), float(rope_base), _ptr(positions), _ptr(pool),
+        pool.shape[0], _ptr(page_table), page_table.shape[1], B, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "mlra_project_append")
+    return workspace
 
 
 def mlra_plan(handle: Handle, seq_lens, pt_stride: int, max_segments: int = 4096, stream=None):

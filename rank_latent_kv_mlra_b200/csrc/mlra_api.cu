@@ -16,6 +16,7 @@
 #include "../../include/mlra.h"
 #include "aux_kernels.cuh"
 #include "common.cuh"
+#include "producer.cuh"
 #include "decode.cuh"
 #include "proj.cuh"
 
@@ -146,6 +147,14 @@ cudaError_t prep_kernel(K kernel, int smem) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                               cudaSharedmemCarveoutMaxShared);
 }
+cudaError_t prep_producer() {
+  cudaError_t e = prep_kernel(mlra_down_proj_kernel<DownShape<16>>, DownShape<16>::SMEM);
+  if (e == cudaSuccess) e = prep_kernel(mlra_down_proj_kernel<DownShape<32>>, DownShape<32>::SMEM);
+  if (e == cudaSuccess) e = prep_kernel(mlra_down_proj_kernel<DownShape<64>>, DownShape<64>::SMEM);
+  if (e == cudaSuccess) e = prep_kernel(mlra_down_proj_kernel<DownShape<128>>, DownShape<128>::SMEM);
+  return e;
+}
+
 template <class Dec>
 cudaError_t prep_decode() {
   return prep_kernel(mlra_decode_kernel<Dec>, Dec::SMEM_BYTES);
@@ -484,6 +493,23 @@ int noalloc_scratch(int dev, void** out) {
 
 }  // namespace
 
+namespace {
+constexpr int kProjSlice = 128;  // d_model columns per down-projection CTA
+size_t project_ws_bytes(const mlra_ctx* h, int batch, int d_model) {
+  const size_t d_out = (size_t)h->cfg.d_c + h->d_r;
+  return 256 + ((size_t)(d_model / kProjSlice) * batch * d_out * 4 + 255) / 256 * 256;
+}
+template <int NT>
+cudaError_t launch_down_proj(const CUtensorMap& mw, const CUtensorMap& mx, const DownParams& dp, int d_out,
+                             int kslices, int batch, cudaStream_t s) {
+  using S = DownShape<NT>;
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t c = launch_cfg(dim3((d_out + 127) / 128, kslices, (batch + NT - 1) / NT), dim3(S::THREADS),
+                                    S::SMEM, s, true, &attr);
+  return cudaLaunchKernelEx(&c, mlra_down_proj_kernel<S>, mw, mx, dp);
+}
+}  // namespace
+
 extern "C" {
 
 int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra_handle* out) {
@@ -566,6 +592,7 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
     default:
       break;
   }
+  if (e == cudaSuccess) e = prep_producer();
   if (e != cudaSuccess) {
     delete h;
     return MLRA_ERR_CUDA;
@@ -640,6 +667,56 @@ int mlra_append_cache(mlra_handle h, void* pool, int num_pages, const int32_t* p
       static_cast<__nv_bfloat16*>(pool), num_pages, page_table, pt_stride, batch, seq_ids, positions, c_new,
       kr_new, in_dtype == MLRA_F32, n_tokens, h->cfg.d_c, h->d_r, status);
   return cudaGetLastError() == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
+}
+
+int mlra_project_workspace_size(mlra_handle h, int batch, int d_model, size_t* bytes) {
+  if (!h || !bytes || batch < 0 || d_model <= 0 || d_model % kProjSlice != 0) return MLRA_ERR_INVALID_ARG;
+  *bytes = project_ws_bytes(h, batch, d_model);
+  return MLRA_OK;
+}
+
+int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w_down, float rope_base,
+                        const int32_t* positions, void* pool, int num_pages, const int32_t* page_table,
+                        int pt_stride, int batch, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h || !x || !w_down || !positions || !pool || !page_table || !workspace) return MLRA_ERR_INVALID_ARG;
+  if (batch < 0 || batch > 65536 || num_pages <= 0 || pt_stride <= 0) return MLRA_ERR_INVALID_ARG;
+  if (d_model <= 0 || d_model % kProjSlice != 0) return MLRA_ERR_INVALID_ARG;
+  const int d_out = h->cfg.d_c + h->d_r;
+  if (d_out % 2 != 0 || h->d_r % 2 != 0) return MLRA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w_down) || reinterpret_cast<uintptr_t>(workspace) % 256 != 0 ||
+      reinterpret_cast<uintptr_t>(pool) % 4 != 0)
+    return MLRA_ERR_INVALID_ARG;
+  if (ws_bytes < project_ws_bytes(h, batch, d_model)) return MLRA_ERR_WORKSPACE;
+  if (batch == 0) return MLRA_OK;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MLRA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nt = nt_for(batch, 128);
+  const int kslices = d_model / kProjSlice;
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, w_down, (uint64_t)d_out, (uint64_t)d_model, (uint64_t)d_model * 2, 128, 64) ||
+      !make_map(&mx, x, (uint64_t)batch, (uint64_t)d_model, (uint64_t)d_model * 2, (uint32_t)nt, 64))
+    return MLRA_ERR_CUDA;
+  int* status = static_cast<int*>(workspace);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
+  DownParams dp = {d_out, batch, part, status, kWaitLimitNs};
+  g_use_pdl = true;
+  cudaError_t e;
+  switch (nt) {
+    case 16: e = launch_down_proj<16>(mw, mx, dp, d_out, kslices, batch, s); break;
+    case 32: e = launch_down_proj<32>(mw, mx, dp, d_out, kslices, batch, s); break;
+    case 64: e = launch_down_proj<64>(mw, mx, dp, d_out, kslices, batch, s); break;
+    default: e = launch_down_proj<128>(mw, mx, dp, d_out, kslices, batch, s); break;
+  }
+  if (e != cudaSuccess) return MLRA_ERR_CUDA;
+  AppendRowParams ap = {part, kslices, batch, h->cfg.d_c, h->d_r, d_out, positions, page_table, pt_stride,
+                        num_pages, static_cast<__nv_bfloat16*>(pool),
+                        std::log2((double)(rope_base > 1.f ? rope_base : 10000.f)), status};
+  const int threads = 256, total = batch * (d_out / 2);
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t c = launch_cfg(dim3((total + threads - 1) / threads), dim3(threads), 0, s, true, &attr);
+  if (cudaLaunchKernelEx(&c, mlra_rope_append_kernel, ap) != cudaSuccess) return MLRA_ERR_CUDA;
+  return MLRA_OK;
 }
 
 int mlra_plan(mlra_handle h, const int32_t* seq_lens, int batch, int pt_stride, int32_t* segments,

@@ -205,3 +205,27 @@ def logical_rows(inputs: dict, b: int) -> torch.Tensor:
     pt = inputs["page_table"][b].to(torch.int64)
     t = torch.arange(n, device=pt.device)
     return inputs["pool"][pt[t // PAGE_SIZE], t % PAGE_SIZE]
+
+
+# The step before decoding (each sequence's new cache row) needs the model width, which the
+# decode workloads do not fix: DeepSeek-V2's hidden size, matching the headline's
+# DeepSeek-V2-like attention shapes.
+PRODUCER_D_MODEL = 5120
+
+
+def make_producer_inputs(w: Workload, inputs: dict, d_model: int = PRODUCER_D_MODEL,
+                         seed: Optional[int] = None) -> dict:
+    """Inputs of the new-row step for workload ``w``'s batch, on the device of ``inputs``:
+    hidden states x [batch][d_model] ~ N(0,1) and w_down [d_c + d_r][d_model] ~
+    N(0,1)/sqrt(d_model) (fan_in = d_model), both bf16, and one position per sequence drawn
+    uniformly from the slots its page-table row covers."""
+    device = inputs["pool"].device
+    s = (w.seed if seed is None else seed) * 31 + 17
+    g = _gen(device, s)
+    x = torch.randn(w.batch, d_model, generator=g, device=device).to(torch.bfloat16)
+    w_down = (torch.randn(w.d_c + w.d_r, d_model, generator=g, device=device) / math.sqrt(d_model)).to(
+        torch.bfloat16)
+    cap = (inputs["page_table"] >= 0).sum(dim=1).to("cpu", torch.int64) * PAGE_SIZE
+    u = torch.rand(w.batch, generator=_gen("cpu", s + 1), dtype=torch.float64)
+    positions = torch.minimum((u * cap).long(), cap - 1).clamp(min=0).to(torch.int32)
+    return {"x": x, "w_down": w_down, "positions": positions.to(device), "d_model": d_model}
