@@ -712,9 +712,10 @@ int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w
   AppendRowParams ap = {part, kslices, batch, h->cfg.d_c, h->d_r, d_out, positions, page_table, pt_stride,
                         num_pages, static_cast<__nv_bfloat16*>(pool),
                         std::log2((double)(rope_base > 1.f ? rope_base : 10000.f)), status};
-  const int threads = 256, total = batch * (d_out / 2);
+  const int total = batch * (d_out / 2);
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3((total + threads - 1) / threads), dim3(threads), 0, s, true, &attr);
+  cudaLaunchConfig_t c = launch_cfg(dim3((total + kAppendPairs - 1) / kAppendPairs),
+                                    dim3(kAppendPairs, kAppendGroups), 0, s, true, &attr);
   if (cudaLaunchKernelEx(&c, mlra_rope_append_kernel, ap) != cudaSuccess) return MLRA_ERR_CUDA;
   return MLRA_OK;
 }

@@ -16,9 +16,9 @@
 //     by TMA, K-major, accumulated in TMEM and written as fp32 partials [slice][b][feature].
 //     Splitting d_model spreads the weight stream (the whole cost: it is read once) over all
 //     SMs.
-//   mlra_rope_append_kernel: one thread per (token, feature pair) sums the slices, rotates the
-//     RoPE pairs (angle in double precision: pos reaches 2^17), rounds to bf16 and stores the
-//     pair into the token's page slot.
+//   mlra_rope_append_kernel: four threads per (token, feature pair) sum the slices, one of them
+//     rotates the RoPE pairs (angle in double precision: pos reaches 2^17), rounds to bf16 and
+//     stores the pair into the token's page slot.
 #pragma once
 
 #include "common.cuh"
@@ -159,37 +159,81 @@ struct AppendRowParams {
   int* status;
 };
 
-__global__ void __launch_bounds__(256) mlra_rope_append_kernel(const AppendRowParams p) {
+// Block (kAppendPairs, kAppendGroups): x = feature pair of one token, y = one of the groups of
+// d_model slices that are summed separately (slices y, y + groups, ...), then combined through
+// shared memory. Loads of one slice by a warp cover 256 contiguous bytes.
+constexpr int kAppendPairs = 64;
+constexpr int kAppendGroups = 4;
+
+__global__ void __launch_bounds__(kAppendPairs * kAppendGroups) mlra_rope_append_kernel(const AppendRowParams p) {
+  __shared__ float2 red[kAppendGroups][kAppendPairs];
   grid_dependency_wait();  // the partials come from the down-projection kernel
   const int pairs = p.d_out / 2;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p.batch * pairs) return;
-  const int b = idx / pairs;
-  const int f0 = 2 * (idx % pairs);
-  const int pos = __ldg(p.positions + b);
-  if (pos < 0 || pos >= p.pt_stride * kPage) {
+  const int idx = blockIdx.x * kAppendPairs + threadIdx.x;
+  const bool live = idx < p.batch * pairs;
+  const int b = live ? idx / pairs : 0;
+  const int f0 = live ? 2 * (idx % pairs) : 0;
+  // the slot's page id is read from a clamped index (always inside the row) so that its load
+  // overlaps the partial sums below; the checks come before the store
+  const int pos = live ? __ldg(p.positions + b) : 0;
+  const int cap = p.pt_stride * kPage;
+  const int page = live ? __ldg(p.page_table + (size_t)b * p.pt_stride + min(max(pos, 0), cap - 1) / kPage) : 0;
+  constexpr int U = 4;  // independent loads in flight per thread
+  const size_t slice = (size_t)p.batch * p.d_out;
+  const float* src = p.part + (size_t)b * p.d_out + f0;
+  float a0[U], a1[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) a0[u] = a1[u] = 0.f;
+  if (live) {
+    int s = threadIdx.y;
+    for (; s + (U - 1) * kAppendGroups < p.kslices; s += U * kAppendGroups) {
+      float2 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        t[u] = __ldcg(reinterpret_cast<const float2*>(src + (size_t)(s + u * kAppendGroups) * slice));
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        a0[u] += t[u].x;
+        a1[u] += t[u].y;
+      }
+    }
+    for (; s < p.kslices; s += kAppendGroups) {
+      const float2 t = __ldcg(reinterpret_cast<const float2*>(src + (size_t)s * slice));
+      a0[0] += t.x;
+      a1[0] += t.y;
+    }
+  }
+  float2 part = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    part.x += a0[u];
+    part.y += a1[u];
+  }
+  red[threadIdx.y][threadIdx.x] = part;
+  __syncthreads();
+  if (threadIdx.y != 0 || !live) return;
+  float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+  for (int g = 0; g < kAppendGroups; ++g) {
+    v0 += red[g][threadIdx.x].x;
+    v1 += red[g][threadIdx.x].y;
+  }
+  if (pos < 0 || pos >= cap) {
     set_status(p.status, kErrSeqLen);
     return;
   }
-  const int page = __ldg(p.page_table + (size_t)b * p.pt_stride + pos / kPage);
   if (page < 0 || page >= p.num_pages) {
     set_status(p.status, kErrPageOob);
     return;
-  }
-  float v0 = 0.f, v1 = 0.f;
-  for (int s = 0; s < p.kslices; ++s) {
-    const float2 t = __ldcg(reinterpret_cast<const float2*>(p.part + ((size_t)s * p.batch + b) * p.d_out + f0));
-    v0 += t.x;
-    v1 += t.y;
   }
   if (f0 >= p.d_c) {
     const int i = (f0 - p.d_c) / 2;
     const double ang = (double)pos * exp2(-2.0 * i / p.d_r * p.log2_base);
     double sn, cs;
     sincos(ang, &sn, &cs);
-    const float c = (float)cs, s = (float)sn;
-    const float r0 = v0 * c - v1 * s;
-    const float r1 = v0 * s + v1 * c;
+    const float cf = (float)cs, sf = (float)sn;
+    const float r0 = v0 * cf - v1 * sf;
+    const float r1 = v0 * sf + v1 * cf;
     v0 = r0;
     v1 = r1;
   }
