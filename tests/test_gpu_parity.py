@@ -221,6 +221,22 @@ def test_empty_and_single_token_sequences():
     G.assert_parity(out.cpu().numpy()[1:3], ref["out"][1:3], "single/short")
 
 
+@pytest.mark.parametrize("batch", [257, 300])
+def test_batches_past_the_warp_plan(batch):
+    """Batches above 256 sequences take the block-wide planner in the decode and combine
+    kernels (and two 128-row batch tiles plus a ragged third in the projections)."""
+    w = W.scaled(SMALL["mlra4_small"], h=32, batch=batch, len_range=(0, 260), seed=60 + batch)
+    inp = W.make_workload(w, device="cuda")
+    hdl = G.make_handle(w, inp)
+    out, lse, ws = G.run_decode(hdl, inp)
+    assert M.mlra_get_status(ws) == 0
+    ref = G.oracle_full(w, inp)
+    G.assert_parity(out.cpu().numpy(), ref["out"], f"batch {batch}")
+    live = ref["lse"] > -1e300
+    assert np.abs(lse.cpu().numpy()[live] - ref["lse"][live]).max() < G.TOL_LSE_ABS
+    assert np.all(np.isneginf(lse.cpu().numpy()[~live]))
+
+
 def test_page_id_out_of_range_is_reported():
     w = SMALL["mlra4_small"]
     inp = W.make_workload(w, device="cuda")
