@@ -19,6 +19,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -109,7 +110,10 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # raw samples go to MLRA_CLOCKS_DIR when set (to keep them), else to a temporary file
+        d = os.environ.get("MLRA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"mlra_clocks_rank{index}_{os.getpid()}.csv")
+        self.keep = bool(os.environ.get("MLRA_CLOCKS_DIR"))
 
     def start(self):
         try:
@@ -145,6 +149,11 @@ class ClockSampler:
                 for n, v in zip(names, p[5:9]):
                     if v.lower() == "active":
                         reasons.add(n)
+        if not self.keep:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),

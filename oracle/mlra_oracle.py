@@ -27,14 +27,14 @@ For head h of group j and a context of n tokens:
 Weights are stored ``[h][d_b][d_h]`` (the ai360xpert code's ``(H, d_c, d_head)`` convention,
 restricted to the head's block of width d_b = d_c/k), so ``K_h[t][d] = sum_c c[t][c] W[h][c][d]``.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * softmax scale: ``1/sqrt(d_h + d_r)`` unless given;
 * k^R is one vector per token, shared by every head and block, cached already rotated;
 * every head has its own q^R_h; RoPE is applied upstream.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (the
 summed-blocks functions by ``tests/test_oracle_summed.py``) except ``plan_segments``, whose rule
-is this build's own (the pages have no split-KV scheme); it is pinned by hand-worked golden
+is not from the pages (they have no split-KV scheme); it is pinned by hand-worked golden
 cases and by invariants (coverage, disjointness, quota).
 """
 from __future__ import annotations

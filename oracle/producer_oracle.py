@@ -17,7 +17,7 @@ What it computes (plain definitions, float64):
 The weights are stored ``w_down[r][d]`` with one row per output feature (latent features
 first, then the RoPE key features), so ``y[r] = sum_d w_down[r][d] x[d]``.
 
-Readings where the pages are silent (listed in the design doc): the rotation follows RoFormer (the
+Readings where the pages are silent: the rotation follows RoFormer (the
 pages cite it; its Section 3.4): feature pairs ``(2i, 2i+1)`` of the RoPE key are rotated by
 the angle ``pos * theta_i`` with ``theta_i = base^(-2i / d_r)``, base 10000 unless given, i.e.
 the pair read as the complex number ``v[2i] + 1j * v[2i+1]`` is multiplied by

@@ -1,6 +1,6 @@
 """GPU parity for the summed-blocks reading (every head attends to every latent block, per-block
 softmax, outputs summed times alpha_attn) through the C ABI, against the float64 oracle's
-``decode_summed``. Reduced sizes compare every element; the full headline-shaped workload
+``decode_summed``. Reduced sizes compare every element; the full-size workload (h = 128, batch 32, context 8192)
 compares sampled heads."""
 import numpy as np
 import pytest

@@ -19,7 +19,7 @@ What a workload holds (all tensors on the requested device):
   ai360xpert "Multi-Head Latent Attention" page stores them ((H, d_c, d_head), "Show Me
   the Code"), restricted to the head's latent block.
 
-Distributions (the pages fix none of them for decode; the readings are listed in the design doc):
+Distributions (the pages fix none of them for decode):
 cache rows and queries N(0,1), weights N(0,1)/sqrt(fan_in) with fan_in = d_c/k (the input
 width of the c -> K/V map). The tiny workload also scales activations by 1/sqrt(width).
 """
@@ -72,10 +72,10 @@ WORKLOADS = {
                  batch=128, len_range=(1024, 32768), seed=4),
         Workload("mla_h128_b128_ragged1k_32k", k=1, h=128, d_h=128, d_c=512, d_r=64,
                  batch=128, len_range=(1024, 32768), seed=4),
-        # the summed-blocks reading of MLRA-4 on the headline's shapes
+        # the summed-blocks reading of MLRA-4 on the h=128, batch-32, context-8192 shapes
         Workload("mlra4sum_h128_b32_n8192", k=4, h=128, d_h=128, d_c=512, d_r=64, batch=32,
                  seq_len=8192, seed=5, summed=True),
-        # One rank's share under 4-way tensor parallelism of the headline's model (h = 128,
+        # One rank's share under 4-way tensor parallelism of the model above (h = 128,
         # d_c = 512, d_r = 64): an MLRA-4 rank holds one block plus the RoPE key and its 32
         # heads; an MLA rank holds the whole latent and 32 heads. Batch 64 keeps either cache
         # larger than L2.
@@ -208,7 +208,7 @@ def logical_rows(inputs: dict, b: int) -> torch.Tensor:
 
 
 # The step before decoding (each sequence's new cache row) needs the model width, which the
-# decode workloads do not fix: DeepSeek-V2's hidden size, matching the headline's
+# decode workloads do not fix: DeepSeek-V2's hidden size, matching the h = 128, d_c = 512
 # DeepSeek-V2-like attention shapes.
 PRODUCER_D_MODEL = 5120
 
