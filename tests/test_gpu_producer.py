@@ -20,6 +20,7 @@ HEAD = W.WORKLOADS["mlra4_h128_b32_n8192"]
 CASES = {
     "small_2slices": (W.scaled(HEAD, batch=3, seq_len=None, len_range=(1, 1500), seed=51), 256),
     "batch100_3slices": (W.scaled(HEAD, batch=100, seq_len=None, len_range=(1, 700), seed=52), 384),
+    "batch300_3tiles": (W.scaled(HEAD, batch=300, seq_len=None, len_range=(1, 300), seed=55), 256),
     "mlra2_small": (W.scaled(W.WORKLOADS["mlra2_h128_b64_n4096"], batch=5, seq_len=None, len_range=(1, 900),
                              seed=53), 512),
     "headline_d5120": (HEAD, W.PRODUCER_D_MODEL),
