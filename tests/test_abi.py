@@ -68,6 +68,8 @@ def test_host_argument_checks_return_codes(lib):
     n = ctypes.c_size_t()
     assert lib.mlra_workspace_size(None, 4, ctypes.byref(n)) == -1
     assert lib.mlra_decode(None, None, 0, None, 0, None, 0, None, 0, None, 0, None, None, 0, None) == -1
+    assert lib.mlra_project_workspace_size(None, 4, 5120, ctypes.byref(n)) == -1
+    assert lib.mlra_project_append(None, None, 5120, None, 0.0, None, None, 0, None, 0, 4, None, 0, None) == -1
     assert lib.mlra_get_info(None, None) == -1
     assert lib.mlra_get_status(None, None) == -1
     lib.mlra_destroy(None)  # NULL-safe
