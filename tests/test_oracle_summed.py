@@ -139,6 +139,17 @@ def test_summed_k1_without_scaling_is_plain_mla():
     np.testing.assert_allclose(got["lse"][:, 0], ref["lse"], rtol=1e-13)
 
 
+def test_default_attn_scale_matches_the_printed_mlra2_table():
+    """alpha_attn when none is given reproduces the MLRA-2 model table (1/2 at k = 2), the only
+    MLRA value the pages print; it is not the GTA table's sqrt(2)/2 = 1/sqrt(2)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "model_tables.json")))
+    row = g["alpha_attn"]["table16_MLRA-2"]
+    assert O.default_attn_scale(row["k"]) == row["value"]
+    assert O.default_attn_scale(row["k"]) != g["alpha_attn"]["table15_GTA"]["value"]
+
+
 def test_summed_empty_sequence():
     rng = np.random.default_rng(9)
     case = _rand_case(rng)
