@@ -78,8 +78,8 @@ typedef struct {
 /* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, heads per block, d_h),
  * heads per block being h/k, or h when blocks_summed:
  *   (32, 16, <=16, 32), (128, 64, <=32 or a multiple of 32, 128),
- *   (256, 64, <=64 or a multiple of 64, 128), (512, 64, a multiple of 32, 128) [k = 1, MLA];
- * blocks_summed with (32, 16, ...) and (128, 64, ...) only; batch <= 4096. */
+ *   (256, 64, <=64 or a multiple of 64, 128), (512, 64, <=64 or a multiple of 64, 128);
+ * blocks_summed with k = 4 and (32, 16, ...) or (128, 64, ...) only; batch <= 4096. */
 
 typedef struct mlra_ctx* mlra_handle;
 
