@@ -38,3 +38,10 @@ def test_decode_flops_partitioned_and_summed():
     # Table 2, MLRA-4: 4 n h (d_c / 4) + 2 n h d_r per device, one block per device, 4 devices
     per_device = 4 * n * ws.h * (ws.d_c // 4) + 2 * n * ws.h * ws.d_r
     assert bench.decode_flops(ws, [n]) == 4 * per_device
+
+
+def test_producer_bytes_match_the_oracle_count():
+    from oracle import producer_oracle as P
+    w = W.WORKLOADS["mlra4_h128_b32_n8192"]
+    for batch, d_model in [(32, 5120), (3, 256), (300, 384)]:
+        assert bench.producer_bytes(w, batch, d_model) == P.bytes_per_step(batch, d_model, w.d_c, w.d_r)
