@@ -71,8 +71,9 @@ typedef struct {
                           the alpha_attn entries of the MLRA index page's model tables point
                           to). Weights are then [k][h][d_b][d_h] and lse is [batch][k*h],
                           block-major (entry j*h + head). */
-  float attn_scale;    /* alpha_attn when blocks_summed: <= 0 selects 1/k (Table 16 prints 1/2
-                          for k = 2; a reading). Ignored otherwise. */
+  float attn_scale;    /* alpha_attn when blocks_summed: <= 0 selects 1/sqrt(k), the values the
+                          MLRA index page's appendix model tables print for MLRA-2 (sqrt(2)/2)
+                          and MLRA-4 (1/2). Ignored otherwise. */
 } mlra_config;
 
 /* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, heads per block, d_h),

@@ -168,13 +168,15 @@ def decode_heads(q, w_uk, w_uv, rows, seq_heads, k, d_r, scale=None):
 # matrices per block, each block under its own softmax, and the head's output is the sum of
 # the k per-block outputs times alpha_attn. This is the reading that the MLRA index page's
 # Table 2 (MLRA-4: 4nh(d_c/4) + 2nh d_h^R FLOPs per device, all h heads on each device's
-# block) and the alpha_attn column of its model tables (Table 16: alpha_attn = 1/2 for
-# MLRA-2) point to; the partitioned reading above is the default one.
+# block) and the alpha_attn column of its model tables (MLRA-2: sqrt(2)/2, MLRA-4: 1/2) point
+# to; the partitioned reading above is the default one.
 # ---------------------------------------------------------------------------------------
 
 def default_attn_scale(k: int) -> float:
-    """alpha_attn when none is given: 1/k (the only value the pages print is 1/2 at k = 2)."""
-    return 1.0 / k
+    """alpha_attn when none is given: 1/sqrt(k). The MLRA index page's appendix model tables
+    print sqrt(2)/2 for MLRA-2 and 1/2 for MLRA-4 (in its extracted text every caption sits
+    below its own table's row, so each of these rows follows the caption of the table before)."""
+    return 1.0 / math.sqrt(k)
 
 
 def decode_summed(q, w_uk, w_uv, pool, page_table, seq_lens, k, d_r, scale=None, attn_scale=None,

@@ -142,7 +142,7 @@ def mlra_create(h: int, d_h: int, d_c: int, d_rope: int, k: int, w_uk: torch.Ten
                 w_uv: torch.Tensor, softmax_scale: float = 0.0, page_size: int = 64,
                 blocks_summed: bool = False, attn_scale: float = 0.0) -> Handle:
     """blocks_summed: every head attends to every block with weights [k][h][d_c/k][d_h] and the
-    per-block outputs are summed times attn_scale (<= 0: 1/k); lse is then [batch][k*h]."""
+    per-block outputs are summed times attn_scale (<= 0: 1/sqrt(k)); lse is then [batch][k*h]."""
     lib = load_library()
     shape = (k, h, d_c // k, d_h) if blocks_summed else (h, d_c // k, d_h)
     for t, n in ((w_uk, "w_uk"), (w_uv, "w_uv")):

@@ -553,7 +553,7 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   h->heads_block = hb;
   h->summed = summed;
   h->vh = summed ? c.k * c.h : c.h;
-  h->alpha = c.attn_scale > 0.f ? c.attn_scale : 1.0f / (float)c.k;
+  h->alpha = c.attn_scale > 0.f ? c.attn_scale : 1.0f / sqrtf((float)c.k);
   h->chunks = (hb + h->np - 1) / h->np;
   h->nsub = c.k * h->chunks;
   h->groups = h->num_sms / h->nsub;

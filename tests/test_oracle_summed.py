@@ -76,9 +76,11 @@ def test_summed_matches_torch_sdpa(k):
     for form in ("absorbed", "explicit"):
         got = _run(case, scale=0.31, attn_scale=0.7, form=form)["out"]
         np.testing.assert_allclose(got, _sdpa_reference(case, 0.31, 0.7), rtol=1e-11, atol=1e-12)
-    # default alpha_attn = 1/k and default scale
+    # default alpha_attn and default scale: the printed model-table values (MLRA-2 sqrt(2)/2,
+    # MLRA-4 1/2), and 1 for a single block (plain MLA has no alpha_attn)
+    printed = {1: 1.0, 2: math.sqrt(2) / 2, 4: 0.5}
     got = _run(case)["out"]
-    ref = _sdpa_reference(case, O.default_scale(case["d_h"], case["d_r"]), 1.0 / k)
+    ref = _sdpa_reference(case, O.default_scale(case["d_h"], case["d_r"]), printed[k])
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
 
 
@@ -139,15 +141,18 @@ def test_summed_k1_without_scaling_is_plain_mla():
     np.testing.assert_allclose(got["lse"][:, 0], ref["lse"], rtol=1e-13)
 
 
-def test_default_attn_scale_matches_the_printed_mlra2_table():
-    """alpha_attn when none is given reproduces the MLRA-2 model table (1/2 at k = 2), the only
-    MLRA value the pages print; it is not the GTA table's sqrt(2)/2 = 1/sqrt(2)."""
+def test_default_attn_scale_matches_the_printed_model_tables():
+    """alpha_attn when none is given reproduces both printed MLRA values: sqrt(2)/2 for MLRA-2
+    and 1/2 for MLRA-4 (the appendix rows that follow the GTA and MLRA-2 captions, each caption
+    sitting below its own table's row in the page text)."""
     import json
     import os
     g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "model_tables.json")))
-    row = g["alpha_attn"]["table16_MLRA-2"]
-    assert O.default_attn_scale(row["k"]) == row["value"]
-    assert O.default_attn_scale(row["k"]) != g["alpha_attn"]["table15_GTA"]["value"]
+    for name in ("MLRA-2", "MLRA-4"):
+        row = g["alpha_attn"][name]
+        assert math.isclose(O.default_attn_scale(row["k"]), row["value"], rel_tol=1e-15), name
+    # 1/k would give the MLRA-2 value 1/2 but the MLRA-4 value 1/4: both rows are needed.
+    assert not math.isclose(1.0 / 4, g["alpha_attn"]["MLRA-4"]["value"])
 
 
 def test_summed_empty_sequence():
