@@ -50,7 +50,12 @@ typedef enum {
   MLRA_ERR_TIMEOUT = -5,       /* device: a pipeline wait passed its time limit */
   MLRA_ERR_WORKSPACE = -6,     /* workspace smaller than mlra_workspace_size */
   MLRA_ERR_SEQ_LEN = -7,       /* device: seq_len < 0 or > pt_stride * page_size */
-  MLRA_ERR_SCRATCH_LIMIT = -8  /* mlra_decode_noalloc: batch too large for its fixed scratch */
+  MLRA_ERR_SCRATCH_LIMIT = -8, /* mlra_decode_noalloc: batch too large for its fixed scratch */
+  MLRA_ERR_DRAIN = -9          /* device: after a wait timed out, copies or MMAs still in flight
+                                  did not finish within the limit either, so shared memory or
+                                  tensor memory may have been released under them. The CUDA
+                                  context may be unusable: stop using it (and the process's
+                                  device state) after this code. Overrides any other code. */
 } mlra_status;
 
 typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype;
@@ -80,7 +85,8 @@ typedef struct {
  * heads per block being h/k, or h when blocks_summed:
  *   (32, 16, <=16, 32), (128, 64, <=32 or a multiple of 32, 128),
  *   (256, 64, <=64 or a multiple of 64, 128), (512, 64, <=64 or a multiple of 64, 128);
- * blocks_summed with k = 4 and (32, 16, ...) or (128, 64, ...) only; batch <= 4096. */
+ * blocks_summed with k = 4 and (32, 16, ...) or (128, 64, ...), or k = 2 and (256, 64, ...);
+ * batch <= 4096. */
 
 typedef struct mlra_ctx* mlra_handle;
 
@@ -109,7 +115,9 @@ int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes);
  *   out        device [batch][h][d_h], dtype out_dtype.
  *   lse        device fp32 [batch][h] natural-log log-sum-exp of the scaled scores, or NULL.
  *   workspace  device, >= mlra_workspace_size(batch) bytes, 256-byte aligned. Its first
- *              4 bytes become this call's status word.
+ *              4 bytes become this call's status word (the first kernel clears it once the
+ *              kernel before it in the stream has finished); the next 8 bytes take errors
+ *              found before that clear, which a later kernel of the call folds into it.
  * Launches three kernels on `stream`: query absorption, split-KV latent attention, and
  * log-sum-exp combine fused with the W^UV up-projection. All three use programmatic
  * dependent launch: the first may begin loading W^UK and setting up while the kernel before
@@ -129,7 +137,10 @@ int mlra_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* po
  *     mlra_workspace_size(batch) <= 16 MiB, i.e. MLRA-4 with 128 heads up to batch 124 on 148 SMs;
  *     larger requests return MLRA_ERR_SCRATCH_LIMIT before any launch.
  *   First call on a device: looks up the array's device address (cudaGetSymbolAddress) with
- *     that device current and keeps it. Make that first call before any stream capture.
+ *     that device current and keeps it. Make that first call before any stream capture. The
+ *     address belongs to the device's current CUDA context: after that context is destroyed
+ *     (cudaDeviceReset, for one) the kept address is stale, so a process that resets a device
+ *     must not call this entry point again on it.
  *   Sharing: every call on a device uses the same array, which keeps the last call's
  *     contents; each call clears the status word it needs at zero. Calls whose kernels
  *     overlap on the GPU (other streams, threads or handles) race on the array: serialise

@@ -33,7 +33,9 @@ Readings where the pages are silent:
 * every head has its own q^R_h; RoPE is applied upstream.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (the
-summed-blocks functions by ``tests/test_oracle_summed.py``) except ``plan_segments``, whose rule
+summed-blocks functions by ``tests/test_oracle_summed.py``; the per-sequence forms
+``decode_sequence`` and ``decode_summed_sequence`` against torch SDPA like the per-head ones)
+except ``plan_segments``, whose rule
 is not from the pages (they have no split-KV scheme); it is pinned by hand-worked golden
 cases and by invariants (coverage, disjointness, quota).
 """
@@ -161,6 +163,84 @@ def decode_heads(q, w_uk, w_uv, rows, seq_heads, k, d_r, scale=None):
         lats.append(lat)
         lses.append(l)
     return np.array(outs), np.array(lats), np.array(lses)
+
+
+def decode_sequence(q_b, w_uk, w_uv, rows, k, d_r, scale=None):
+    """Absorbed-form result for EVERY head of one sequence whose rows are given, with the
+    heads of each latent block stacked so that one matrix product serves them all (used for
+    the elementwise checks at full size, where one head at a time would re-read the rows h
+    times). Same definitions as ``attend_head_absorbed``; for block j and its heads G_j:
+
+      Q~_j = [(W^UK_h)^T q^C_h]_{h in G_j}                      [|G_j|][d_b]
+      S_j  = scale * (c_j Q~_j^T + k^R (Q^R_j)^T)               [n][|G_j|]
+      P_j  = softmax of each column of S_j;  lse_h = log sum_t exp(S_j[t][h])
+      o~_h = (P_j^T c_j)[h];  o_h = W^UV_h o~_h
+
+    q_b: [h][d_h + d_r]; w_uk, w_uv: [h][d_b][d_h]; rows: [n][d_c + d_r].
+    Returns (out [h][d_h], latent [h][d_b], lse [h]); n = 0 gives zeros and -inf."""
+    q_b = np.asarray(q_b, dtype=np.float64)
+    w_uk = np.asarray(w_uk, dtype=np.float64)
+    w_uv = np.asarray(w_uv, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.float64)
+    h, qw = q_b.shape
+    d_h = qw - d_r
+    d_b = w_uk.shape[1]
+    d_c = d_b * k
+    if scale is None:
+        scale = default_scale(d_h, d_r)
+    out = np.zeros((h, d_h))
+    latent = np.zeros((h, d_b))
+    lse = np.full(h, -np.inf)
+    if rows.shape[0] == 0:
+        return out, latent, lse
+    hb = h // k
+    for j in range(k):
+        g = slice(j * hb, (j + 1) * hb)
+        c_j, kr = _split(rows, j, d_c, k)
+        q_lat = np.einsum("hcd,hd->hc", w_uk[g], q_b[g, :d_h])      # [hb][d_b]
+        S = scale * (c_j @ q_lat.T + kr @ q_b[g, d_h:].T)          # [n][hb]
+        m = S.max(axis=0)
+        E = np.exp(S - m)
+        l = E.sum(axis=0)
+        P = E / l
+        lse[g] = m + np.log(l)
+        latent[g] = P.T @ c_j                                      # [hb][d_b]
+        out[g] = np.einsum("hc,hcd->hd", latent[g], w_uv[g])
+    return out, latent, lse
+
+
+def decode_summed_sequence(q_b, w_uk, w_uv, rows, k, d_r, scale=None, attn_scale=None):
+    """``decode_summed`` for every head of one sequence whose rows are given, each block's
+    heads stacked into one matrix product (as in ``decode_sequence``, but every head sees
+    every block through its own W^UK_{j,h}, W^UV_{j,h}). w_uk, w_uv: [k][h][d_b][d_h].
+    Returns (out [h][d_h], lse [k][h])."""
+    q_b = np.asarray(q_b, dtype=np.float64)
+    w_uk = np.asarray(w_uk, dtype=np.float64)
+    w_uv = np.asarray(w_uv, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.float64)
+    h, qw = q_b.shape
+    d_h = qw - d_r
+    d_b = w_uk.shape[2]
+    d_c = d_b * k
+    if scale is None:
+        scale = default_scale(d_h, d_r)
+    if attn_scale is None:
+        attn_scale = default_attn_scale(k)
+    out = np.zeros((h, d_h))
+    lse = np.full((k, h), -np.inf)
+    if rows.shape[0] == 0:
+        return out, lse
+    for j in range(k):
+        c_j, kr = _split(rows, j, d_c, k)
+        q_lat = np.einsum("hcd,hd->hc", w_uk[j], q_b[:, :d_h])
+        S = scale * (c_j @ q_lat.T + kr @ q_b[:, d_h:].T)
+        m = S.max(axis=0)
+        E = np.exp(S - m)
+        l = E.sum(axis=0)
+        lse[j] = m + np.log(l)
+        lat = (E / l).T @ c_j
+        out += attn_scale * np.einsum("hc,hcd->hd", lat, w_uv[j])
+    return out, lse
 
 
 # ---------------------------------------------------------------------------------------

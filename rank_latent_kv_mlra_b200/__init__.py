@@ -87,7 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mlra_get_status.argtypes = [P, ctypes.POINTER(I)]
     lib.mlra_status_string.argtypes = [I]
     lib.mlra_status_string.restype = ctypes.c_char_p
-    lib.mlra_test_decode_stalled.argtypes = [P, P, I, P, I, P, I, P, I, P, P, S, ctypes.c_ulonglong, P]
+    lib.mlra_test_decode_stalled.argtypes = [P, P, I, P, I, P, I, P, I, P, P, S, ctypes.c_ulonglong, I, P]
     _lib = lib
     return lib
 
@@ -341,10 +341,11 @@ def mlra_status_string(code: int) -> str:
 
 
 def mlra_test_decode_stalled(handle: Handle, q, pool, page_table, seq_lens, out, workspace,
-                             wait_limit_ns: int, stream=None):
-    """Test hook: a decode whose producer withholds its first tile (see mlra_api.cu)."""
+                             wait_limit_ns: int, where: int = 1, stream=None):
+    """Test hook: a decode with one wait made to run out (where = 1: the decode kernel's
+    producer withholds its first tile; 2: one absorb CTA never issues its MMA)."""
     B = _decode_common(handle, q, pool, page_table, seq_lens, workspace)
     _check(load_library().mlra_test_decode_stalled(
         handle.ptr, _ptr(q), _dtype(q), _ptr(pool), pool.shape[0], _ptr(page_table),
         page_table.shape[1], _ptr(seq_lens), B, _ptr(out), _ptr(workspace), workspace.numel(),
-        wait_limit_ns, _stream(stream)), "mlra_test_decode_stalled")
+        wait_limit_ns, where, _stream(stream)), "mlra_test_decode_stalled")

@@ -14,10 +14,38 @@ constexpr int kPage = 64;    // tokens per cache page
 constexpr int kTile = 128;   // tokens per decode tile (two pages, the MMA M extent)
 
 // Device status codes (same values as mlra_status).
-enum : int { kOk = 0, kErrPageOob = -4, kErrTimeout = -5, kErrSeqLen = -7 };
+enum : int { kOk = 0, kErrPageOob = -4, kErrTimeout = -5, kErrSeqLen = -7, kErrDrain = -9 };
 
+// First error wins.
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
+}
+// A failed teardown drain overrides any other code: after it the context may be unusable.
+__device__ __forceinline__ void force_status(int* status, int code) {
+  if (status != nullptr) atomicExch(status, code);
+}
+
+// Errors found while the call's status word may not yet be cleared. The first kernel of a
+// call clears the status word from one CTA after the previous kernel in the stream has
+// finished; its other CTAs may fail before that clear. They never write the status word:
+// they store the call's tag (a number unique to each host call, never 0) into a tag word of
+// the workspace, one word per error kind, and a later kernel of the same call, which runs
+// after the first has completed, turns a matching tag into the status code. A tag left in
+// the word by an earlier call never matches. tags[0]: pipeline wait timed out; tags[1]:
+// teardown drain failed.
+struct EarlyTags {
+  unsigned* words;  // 2 words in the call's workspace
+  unsigned tag;     // this call's tag
+};
+__device__ __forceinline__ void report_early(const EarlyTags& t, int which) {
+  if (t.words != nullptr) atomicExch(t.words + which, t.tag);
+}
+// Called by one thread of a later kernel of the same call, after griddepcontrol.wait.
+__device__ __forceinline__ void fold_early(const EarlyTags& t, int* status) {
+  if (t.words == nullptr) return;
+  const unsigned* w = t.words;
+  if (*reinterpret_cast<const volatile unsigned*>(w + 1) == t.tag) force_status(status, kErrDrain);
+  else if (*reinterpret_cast<const volatile unsigned*>(w) == t.tag) set_status(status, kErrTimeout);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

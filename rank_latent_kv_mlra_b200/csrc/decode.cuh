@@ -132,8 +132,9 @@ struct DecodeParams {
   float* o_part;    // [slots][h][DB] fp32, normalised partial latent outputs
   float* lse_part;  // [slots][h] fp32, log2-domain log-sum-exp
   int* status;
+  EarlyTags tags;    // errors of the absorb kernel (folded in by CTA 0)
   unsigned long long wait_limit_ns;
-  int inject_stall;  // test hook: the producer withholds its first tile
+  int inject_stall;  // test hook: 1 = the producer withholds its first tile
 };
 
 // Reduce N per-head values across the 32 lanes of a warp and scatter the results: afterwards
@@ -236,6 +237,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
   int* plan_err = misc + 2;
   int* scratch = misc + 8;  // 40 ints for the planner
   volatile int* plan_words = misc + 48;  // segment count and resume point of the first list
+  volatile int* drain_err = misc + 3;     // a teardown drain ran out of time
 
   const int warp = warp_id(), lane = lane_id();
   const int group = blockIdx.x / p.nsub;
@@ -268,6 +270,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
     mbar_init(&mmadone_bar[1], 1);
     *abort_flag = 0;
     *plan_err = 0;
+    *drain_err = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             for (int g = 0; g < Sh::NG && ok; ++g) {
               const int gi = st * Sh::NG + g;
               ok = mbar_wait(&empty_bar[gi], ph ^ 1, abort_flag, p.wait_limit_ns);
-              if (ok && !(p.inject_stall && it == 0)) {
+              if (ok && !(p.inject_stall == 1 && it == 0)) {
                 if (g == 0) MLRA_TRACE_POINT(1, 8 + min((int)it, 31));
                 mbar_arrive_expect_tx(&full_bar[gi], npg * Sh::group_tx(g));
                 issued_mask |= 1u << gi;
@@ -776,18 +779,26 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
     // wait for the last issued load of every (stage, group) (completed loads return at once)
     for (int gi = 0; gi < STAGES * Sh::NG; ++gi) {
       if (!(issued_mask & (1u << gi))) continue;
-      mbar_wait_drain(&full_bar[gi], (issued_phase >> gi) & 1, p.wait_limit_ns);
+      if (!mbar_wait_drain(&full_bar[gi], (issued_phase >> gi) & 1, p.wait_limit_ns)) *drain_err = 1;
     }
   }
   if (warp == 1 || warp == Sh::PV_WARP) {
     uint64_t* done = &mmadone_bar[warp == 1 ? 0 : 1];
     if (lane == 0) umma_commit(done);
     __syncwarp();
-    mbar_wait_drain(done, 0, p.wait_limit_ns);
+    if (!mbar_wait_drain(done, 0, p.wait_limit_ns) && lane == 0) *drain_err = 1;
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
+  if (threadIdx.x == 0) {
+    // Every CTA waits for the absorb kernel before it exits (a CTA without tiles never did),
+    // so this grid completes only after the absorb grid, and the status word it cleared is
+    // not written by this call's later kernels before the clear.
+    grid_dependency_wait();
+    if (blockIdx.x == 0) fold_early(p.tags, p.status);
+    if (*abort_flag) set_status(p.status, kErrTimeout);
+    if (*drain_err) force_status(p.status, kErrDrain);
+  }
   if (threadIdx.x == 0) MLRA_TRACE_POINT(1, 201);
   if (warp == 1) {
     tc_fence_after();

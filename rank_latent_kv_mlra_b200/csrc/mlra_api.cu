@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -28,7 +29,7 @@ namespace {
 // Compiled kernel set. A variant fixes (d_b, d_rope, heads per CTA, d_h) and the decode
 // kernel's shared-memory pipeline.
 // ---------------------------------------------------------------------------------------
-enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kMlra4Sum = 4, kNumVariants };
+enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kMlra4Sum = 4, kMlra2Sum = 5, kNumVariants };
 
 using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 // P is written over each stage's RoPE columns, which leaves room for two query buffers (the
@@ -50,7 +51,8 @@ struct VariantDims {
   int d_b, d_r, np, d_h;
 };
 constexpr VariantDims kDims[kNumVariants] = {
-    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 64, 128}, {128, 64, 64, 128}};
+    {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 64, 128}, {128, 64, 64, 128},
+    {256, 64, 64, 128}};
 
 // Largest batch tile of the projection kernels: at d_b = 512 a 128-row tile of the merged
 // latent plus W^UV^T would need 256 KB of shared memory.
@@ -110,6 +112,14 @@ bool make_q_map(CUtensorMap* m, const void* q, uint64_t batch, uint64_t heads, u
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A number unique to each host call that launches kernels (never 0): see EarlyTags.
+std::atomic<unsigned> g_call_tag{0};
+unsigned next_call_tag() {
+  unsigned t = ++g_call_tag;
+  while (t == 0) t = ++g_call_tag;
+  return t;
 }
 
 int nt_for(int batch, int max_nt) {
@@ -362,8 +372,12 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   pp.q_heads = h->cfg.h;
   pp.out_heads = h->cfg.h;
   pp.out_scale = h->summed ? h->alpha : 1.f;
+  // the status word's first 4 bytes; the next two words take early errors by call tag
+  const EarlyTags tags = {reinterpret_cast<unsigned*>(w.status) + 1, next_call_tag()};
   pp.status = w.status;
+  pp.tags = tags;
   pp.wait_limit_ns = wait_limit_ns;
+  pp.inject_stall = inject_stall;
 
   DecodeParams dp = {};
   dp.seq_lens = seq_lens;
@@ -381,6 +395,7 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   dp.o_part = w.o_part;
   dp.lse_part = w.lse_part;
   dp.status = w.status;
+  dp.tags = tags;
   dp.wait_limit_ns = wait_limit_ns;
   dp.inject_stall = inject_stall;
 
@@ -433,6 +448,17 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
         e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
                    : dispatch_uproj<256, 128, false>(h, pp, batch, s);
       break;
+    case kMlra2Sum:
+      // every head on each of the two 256-wide blocks: the MLRA-2 decode kernel over 2h
+      // virtual heads, then one GEMM over the stacked 512-wide merged latents
+      e = dispatch_absorb<256, 128>(h, pp, batch, s);
+      rec(1);
+      if (e == cudaSuccess) e = launch_decode<DecMlra2>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<512, 128, false, 2>(h, pp, batch, s);
+      break;
     case kMla:
       e = dispatch_absorb<512, 128>(h, pp, batch, s);
       rec(1);
@@ -461,8 +487,8 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
 // kNoAllocScratchBytes is the whole array; every GPU that loads this library holds it until
 // the process exits. It covers mlra_workspace_size(batch) for MLRA-4 with 128 heads up to
 // batch 124 on a 148-SM GPU. All calls on a device share the one array and it keeps what the
-// last call left there, so each call clears the status word (every other byte the kernels
-// read is written earlier in the same call). Calls whose kernels overlap on the GPU (other
+// last call left there: the status word is cleared by the call's first kernel, as in
+// mlra_decode, and every other byte the kernels read is written earlier in the same call. Calls whose kernels overlap on the GPU (other
 // streams, other threads, other handles on the same device) race on it.
 // ---------------------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
@@ -530,9 +556,11 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
         (hb <= kDims[v].np || hb % kDims[v].np == 0))
       var = v;
   if (var < 0) return MLRA_ERR_UNSUPPORTED;
-  // summed blocks: the combine's GEMM runs over k*d_b, compiled for these two shapes
-  if (summed && !((var == kMlra4 && c.k == 4) || (var == kTiny && c.k == 4))) return MLRA_ERR_UNSUPPORTED;
+  // summed blocks: the combine's GEMM runs over k*d_b, compiled for these three shapes
+  if (summed && !((var == kMlra4 && c.k == 4) || (var == kTiny && c.k == 4) || (var == kMlra2 && c.k == 2)))
+    return MLRA_ERR_UNSUPPORTED;
   if (summed && var == kMlra4) var = kMlra4Sum;
+  if (summed && var == kMlra2) var = kMlra2Sum;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLRA_ERR_CUDA;
@@ -589,6 +617,12 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
       if (e == cudaSuccess) e = prep_proj_all<512, 128>();
       h->stages = DecMla::STAGES;
       break;
+    case kMlra2Sum:
+      e = prep_decode<DecMlra2>();
+      if (e == cudaSuccess) e = prep_proj_all<256, 128>();
+      if (e == cudaSuccess) e = prep_proj_sum<512, 128, 2>();
+      h->stages = DecMlra2::STAGES;
+      break;
     default:
       break;
   }
@@ -638,7 +672,6 @@ int mlra_decode_noalloc(mlra_handle h, const void* q, mlra_dtype q_dtype, const 
   int rc = noalloc_scratch(dev, &scratch);
   if (rc != MLRA_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return MLRA_ERR_CUDA;
   rc = run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, out_dtype, lse,
                   nullptr, scratch, kNoAllocScratchBytes, stream, 0, kWaitLimitNs);
   if (rc != MLRA_OK) return rc;
@@ -699,7 +732,8 @@ int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w
     return MLRA_ERR_CUDA;
   int* status = static_cast<int*>(workspace);
   float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
-  DownParams dp = {d_out, batch, part, status, kWaitLimitNs};
+  const EarlyTags tags = {reinterpret_cast<unsigned*>(status) + 1, next_call_tag()};
+  DownParams dp = {d_out, batch, part, status, tags, kWaitLimitNs};
   g_use_pdl = true;
   cudaError_t e;
   switch (nt) {
@@ -711,7 +745,7 @@ int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w
   if (e != cudaSuccess) return MLRA_ERR_CUDA;
   AppendRowParams ap = {part, kslices, batch, h->cfg.d_c, h->d_r, d_out, positions, page_table, pt_stride,
                         num_pages, static_cast<__nv_bfloat16*>(pool),
-                        std::log2((double)(rope_base > 1.f ? rope_base : 10000.f)), status};
+                        std::log2((double)(rope_base > 1.f ? rope_base : 10000.f)), status, tags};
   const int total = batch * (d_out / 2);
   cudaLaunchAttribute attr;
   cudaLaunchConfig_t c = launch_cfg(dim3((total + kAppendPairs - 1) / kAppendPairs),
@@ -760,6 +794,7 @@ const char* mlra_status_string(int code) {
     case MLRA_ERR_WORKSPACE: return "workspace too small";
     case MLRA_ERR_SEQ_LEN: return "sequence length outside its page-table row";
     case MLRA_ERR_SCRATCH_LIMIT: return "batch needs more than the 16 MiB fixed scratch of mlra_decode_noalloc";
+    case MLRA_ERR_DRAIN: return "in-flight device copies or MMAs did not finish after a failed wait: stop using this CUDA context";
     default: return "unknown status";
   }
 }
@@ -776,15 +811,18 @@ int mlra_decode_profiled(mlra_handle h, const void* q, mlra_dtype q_dtype, const
                     lse, nullptr, workspace, ws_bytes, stream, 0, kWaitLimitNs, events);
 }
 
-// Test hook (not in the public header): a decode whose producer withholds its first tile, so
-// the consumer's bounded wait runs out after `wait_limit_ns` and the status word reports
-// MLRA_ERR_TIMEOUT. Used to check that a stalled pipeline ends with an error, not a hang.
+// Test hook (not in the public header): a decode with one wait made to run out after
+// `wait_limit_ns`, so the status word must report MLRA_ERR_TIMEOUT. where = 1: the decode
+// kernel's producer withholds each CTA's first tile; where = 2: absorb CTA (1, 0) never issues
+// its MMA (an error raised by a CTA other than the one that clears the status word). Used to
+// check that a stalled pipeline ends with an error, not a hang, and that the error survives.
 int mlra_test_decode_stalled(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* pool,
                              int num_pages, const int32_t* page_table, int pt_stride,
                              const int32_t* seq_lens, int batch, void* out, void* workspace,
-                             size_t ws_bytes, unsigned long long wait_limit_ns, void* stream) {
+                             size_t ws_bytes, unsigned long long wait_limit_ns, int where, void* stream) {
+  if (where != 1 && where != 2) return MLRA_ERR_INVALID_ARG;
   return run_decode(h, q, q_dtype, pool, num_pages, page_table, pt_stride, seq_lens, batch, out, MLRA_F32,
-                    nullptr, nullptr, workspace, ws_bytes, stream, 1, wait_limit_ns);
+                    nullptr, nullptr, workspace, ws_bytes, stream, where, wait_limit_ns);
 }
 
 #ifdef MLRA_TRACE

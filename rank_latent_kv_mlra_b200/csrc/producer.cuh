@@ -29,7 +29,8 @@ struct DownParams {
   int d_out;    // d_c + d_r
   int batch;
   float* part;  // [kslices][batch][d_out] fp32
-  int* status;
+  int* status;  // cleared by CTA (0, 0, 0); written by the append kernel
+  EarlyTags tags;  // this kernel's errors (the append kernel folds them into status)
   unsigned long long wait_limit_ns;
 };
 
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(Sh::THREADS)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int mt = blockIdx.x, ks = blockIdx.y, n0 = blockIdx.z * NT;
   const int warp = warp_id(), lane = lane_id();
+  bool mma_issued = false;  // (warp 0) the MMA went out: its commit is drained at teardown
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(Sh::THREADS)
         umma_commit(&bars[1]);
       }
       __syncwarp();
+      mma_issued = true;
     }
   }
   const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
@@ -135,10 +138,16 @@ __global__ void __launch_bounds__(Sh::THREADS)
     }
   }
   // drain before releasing TMEM and shared memory
-  if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+  bool drained = true;
+  if (threadIdx.x == 0) {
+    drained = mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+    if (mma_issued) drained = mbar_wait_drain(&bars[1], 0, p.wait_limit_ns) && drained;
+  }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
+  // this kernel may fail before CTA (0, 0, 0) has cleared the status word: report by tag
+  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, 0);
+  if (threadIdx.x == 0 && !drained) report_early(p.tags, 1);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM);
@@ -157,6 +166,7 @@ struct AppendRowParams {
   __nv_bfloat16* pool;    // [num_pages][64][d_out]
   double log2_base;       // log2 of the RoPE base
   int* status;
+  EarlyTags tags;         // the down-projection kernel's errors, folded in by block 0
 };
 
 // Block (kAppendPairs, kAppendGroups): x = feature pair of one token, y = one of the groups of
@@ -168,6 +178,7 @@ constexpr int kAppendGroups = 4;
 __global__ void __launch_bounds__(kAppendPairs * kAppendGroups) mlra_rope_append_kernel(const AppendRowParams p) {
   __shared__ float2 red[kAppendGroups][kAppendPairs];
   grid_dependency_wait();  // the partials come from the down-projection kernel
+  if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) fold_early(p.tags, p.status);
   const int pairs = p.d_out / 2;
   const int idx = blockIdx.x * kAppendPairs + threadIdx.x;
   const bool live = idx < p.batch * pairs;

@@ -55,8 +55,10 @@ struct ProjParams {
   int q_heads;        // heads of the query rows (head v reads query row v % q_heads)
   int out_heads;      // heads of the output rows
   float out_scale;    // alpha_attn when the blocks are summed, else 1
-  int* status;
+  int* status;        // cleared by absorb CTA (0, 0); written by the combine kernel
+  EarlyTags tags;     // absorb errors (the decode kernel folds them into status)
   unsigned long long wait_limit_ns;
+  int inject_stall;   // test hook: 2 = absorb CTA (1, 0) never issues its MMA, so its wait runs out
 };
 
 template <int DB_, int DH_, int NT_>
@@ -120,6 +122,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int n0 = blockIdx.y * NT;
   const int warp = warp_id(), lane = lane_id();
   const int qw = DB + p.d_r;
+  bool mma_issued = false;  // (warp 0) the MMA went out: its commit is drained at teardown
   const int hb = head % p.heads_block;
   const int blk = head / p.heads_block;
   const int sub = blk * p.chunks + hb / p.np;
@@ -240,9 +243,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __syncthreads();
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 2);
 
+  const bool stall = p.inject_stall == 2 && blockIdx.x == 1 && blockIdx.y == 0;
   if (warp == 0) {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, abort_flag, p.wait_limit_ns));
-    if (ok) {
+    if (ok && !stall) {
       tc_fence_after();
       if (lane == 0) {
         MLRA_TRACE_POINT(0, 3);
@@ -262,6 +266,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         umma_commit(&bars[1]);
       }
       __syncwarp();
+      mma_issued = true;
     }
   }
   if (tma_q && warp != 0) {
@@ -330,10 +335,16 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   }
   // drain before releasing TMEM and shared memory
   if (threadIdx.x == 0) MLRA_TRACE_POINT(0, 5);
-  if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+  bool drained = true;
+  if (threadIdx.x == 0) {
+    drained = mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+    if (mma_issued) drained = mbar_wait_drain(&bars[1], 0, p.wait_limit_ns) && drained;
+  }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kErrTimeout);
+  // this kernel may fail before CTA (0, 0) has cleared the status word: report by tag
+  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, 0);
+  if (threadIdx.x == 0 && !drained) report_early(p.tags, 1);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM1);
@@ -564,6 +575,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 3);
   if (err) atomicOr(err_flag, 1);
 
+  bool mma_issued = false;  // (warp 0) the MMA went out: its commit is drained at teardown
   if constexpr (!LATENT_ONLY) {
     fence_proxy_async_smem();
     __syncthreads();
@@ -586,6 +598,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           umma_commit(&bars[1]);
         }
         __syncwarp();
+        mma_issued = true;
       }
     }
     const bool ok = mbar_wait(&bars[1], 0, abort_flag, p.wait_limit_ns);
@@ -629,13 +642,17 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       }
     }
     if (threadIdx.x == 0) MLRA_TRACE_POINT(2, 6);
-    if (threadIdx.x == 0) mbar_wait_drain(&bars[0], 0, p.wait_limit_ns);
+    if (threadIdx.x == 0) {
+      if (!mbar_wait_drain(&bars[0], 0, p.wait_limit_ns)) atomicOr(err_flag, 2);
+      if (mma_issued && !mbar_wait_drain(&bars[1], 0, p.wait_limit_ns)) atomicOr(err_flag, 2);
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    if (*err_flag) set_status(p.status, kErrSeqLen);
+    if (*err_flag & 1) set_status(p.status, kErrSeqLen);
     if (*abort_flag) set_status(p.status, kErrTimeout);
+    if (*err_flag & 2) force_status(p.status, kErrDrain);
   }
   if (!LATENT_ONLY && warp == 0) {
     tc_fence_after();

@@ -95,6 +95,53 @@ def test_matches_torch_sdpa_on_reconstructed_heads(k):
         np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
 
 
+def _per_sequence(case, scale):
+    """decode_sequence over every sequence of a case (rows gathered like the GPU tests do)."""
+    B, h = case["q"].shape[:2]
+    out = np.zeros((B, h, case["d_h"]))
+    lse = np.zeros((B, h))
+    for b in range(B):
+        rows = O.gather_rows(case["pool"], case["page_table"], b, int(case["seq_lens"][b]))
+        out[b], _, lse[b] = O.decode_sequence(case["q"][b], case["w_uk"], case["w_uv"], rows, case["k"],
+                                              case["d_r"], scale=scale)
+    return out, lse
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+def test_per_sequence_form_matches_torch_sdpa(k):
+    """The all-heads-at-once form against the same independent SDPA reference, and its lse
+    against scipy's logsumexp of explicitly formed scores."""
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(20 + k)
+    case = _rand_case(rng, k=k, d_b=96 // k, lens=(1, 200))
+    out, lse = _per_sequence(case, 0.29)
+    np.testing.assert_allclose(out, _sdpa_reference(case, 0.29), rtol=1e-11, atol=1e-12)
+    d_h, d_c, h = case["d_h"], case["d_c"], case["h"]
+    d_b = d_c // k
+    for b in range(2):
+        rows = O.gather_rows(case["pool"], case["page_table"], b, int(case["seq_lens"][b]))
+        for hd in range(h):
+            j = hd // (h // k)
+            s = 0.29 * (rows[:, j * d_b:(j + 1) * d_b] @ case["w_uk"][hd] @ case["q"][b, hd, :d_h]
+                        + rows[:, d_c:] @ case["q"][b, hd, d_h:])
+            assert abs(lse[b, hd] - logsumexp(s)) < 1e-12
+
+
+def test_per_sequence_form_empty_sequence():
+    rng = np.random.default_rng(5)
+    case = _rand_case(rng)
+    out, lat, lse = O.decode_sequence(case["q"][0], case["w_uk"], case["w_uv"], np.zeros((0, case["d_c"] + 8)),
+                                      case["k"], case["d_r"])
+    assert np.all(out == 0) and np.all(lat == 0) and np.all(np.isneginf(lse))
+
+
+def test_planted_mistake_in_per_sequence_form_is_caught(monkeypatch):
+    real_split = O._split
+    monkeypatch.setattr(O, "_split", lambda rows, j, d_c, k: real_split(rows, (j + 1) % k, d_c, k))
+    with pytest.raises(AssertionError):
+        test_per_sequence_form_matches_torch_sdpa(4)
+
+
 def test_absorbed_equals_explicit_reconstruction():
     """Absorption is exact (ai360xpert: reconstruction is exact; lesty.tech section 5)."""
     rng = np.random.default_rng(1)

@@ -84,6 +84,23 @@ def test_summed_matches_torch_sdpa(k):
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("k", [2, 4])
+def test_summed_per_sequence_form_matches_torch_sdpa(k):
+    """decode_summed_sequence (every head of a sequence at once) against the independent SDPA
+    reference, at a given and at the default alpha_attn."""
+    rng = np.random.default_rng(60 + k)
+    case = _rand_case(rng, k=k, d_b=96 // k, lens=(3, 190))
+    printed = {2: math.sqrt(2) / 2, 4: 0.5}
+    for alpha in (0.8, None):
+        ref = _sdpa_reference(case, 0.33, printed[k] if alpha is None else alpha)
+        for b in range(2):
+            rows = _rows(case, b)
+            out, lse = O.decode_summed_sequence(case["q"][b], case["w_uk"], case["w_uv"], rows, k, case["d_r"],
+                                                scale=0.33, attn_scale=alpha)
+            np.testing.assert_allclose(out, ref[b], rtol=1e-11, atol=1e-12)
+            assert lse.shape == (k, case["h"])
+
+
 def test_summed_lse_per_block_matches_logsumexp():
     rng = np.random.default_rng(3)
     case = _rand_case(rng)

@@ -75,6 +75,10 @@ WORKLOADS = {
         # the summed-blocks reading of MLRA-4 on the h=128, batch-32, context-8192 shapes
         Workload("mlra4sum_h128_b32_n8192", k=4, h=128, d_h=128, d_c=512, d_r=64, batch=32,
                  seq_len=8192, seed=5, summed=True),
+        # the summed-blocks reading of MLRA-2 (two blocks of 256, all 128 heads on each) on
+        # the batch-64, context-4096 shapes
+        Workload("mlra2sum_h128_b64_n4096", k=2, h=128, d_h=128, d_c=512, d_r=64, batch=64,
+                 seq_len=4096, seed=7, summed=True),
         # One rank's share under 4-way tensor parallelism of the model above (h = 128,
         # d_c = 512, d_r = 64): an MLRA-4 rank holds one block plus the RoPE key and its 32
         # heads; an MLA rank holds the whole latent and 32 heads. Batch 64 keeps either cache
