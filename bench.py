@@ -101,63 +101,116 @@ def recorded_traffic(workload_name):
 
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    """SM clock and throttle reasons sampled during the measured legs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Read-only NVML queries from a background thread every ~1 ms (the decode step takes tens of
+    microseconds, so the sampler runs from the first warm-up step to the end of the profiled
+    leg, and `under_load` counts the samples taken while the GPU was not idle); `nvidia-smi
+    -lms 100` in a subprocess is the fallback when NVML cannot be loaded."""
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        # raw samples go to MLRA_CLOCKS_DIR when set (to keep them), else to a temporary file
-        d = os.environ.get("MLRA_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(d, f"mlra_clocks_rank{index}_{os.getpid()}.csv")
-        self.keep = bool(os.environ.get("MLRA_CLOCKS_DIR"))
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.samples = []
+        self.max_mhz = None
+        self.thread = None
+        self.stop_flag = False
+        self.smi = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        bus = torch.cuda.get_device_properties(self.device).pci_bus_id  # e.g. 0000:1B:00.0
+        try:
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        return pynvml, h
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            nv, h = self._nvml_handle()
         except Exception:
-            self.proc = None
+            self._start_smi()
+            return
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        bits = {name: getattr(nv, attr) for name, attr in self.REASONS}
+        idle = nv.nvmlClocksEventReasonGpuIdle
+
+        def run():
+            while not self.stop_flag:
+                try:
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    self.samples.append((mhz, r & idle != 0, [n for n, b in bits.items() if r & b]))
+                except Exception:
+                    pass
+                time.sleep(0.001)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.gpu_idle,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = tempfile.TemporaryFile(mode="w+")
+            idx = self.device.index or 0
+            self.smi = subprocess.Popen(["nvidia-smi", f"--id={idx}", f"--query-gpu={fields}",
+                                         "--format=csv,noheader,nounits", "-lms", "100"],
+                                        stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.smi = None
+
+    def _stop_smi(self):
+        self.smi.terminate()
+        try:
+            self.smi.wait(timeout=5)
+        except Exception:
+            self.smi.kill()
+        self.fh.seek(0)
+        names = [n for n, _ in self.REASONS]
+        for line in self.fh:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 7:
+                continue
+            try:
+                mhz, self.max_mhz = float(p[0]), float(p[1])
+            except ValueError:
+                continue
+            self.samples.append((mhz, p[2].lower() == "active",
+                                 [n for n, v in zip(names, p[3:7]) if v.lower() == "active"]))
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+        elif self.smi is not None:
+            self._stop_smi()
+        else:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                p = [x.strip() for x in line.split(",")]
-                if len(p) < 9:
-                    continue
-                try:
-                    sm.append(float(p[1]))
-                    mx = float(p[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, p[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        if not self.keep:
-            try:
-                os.remove(self.path)
-            except OSError:
-                pass
-        if not sm:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        load = [s for s in self.samples if not s[1]] or self.samples
+        reasons = sorted({r for s in load for r in s[2]})
+        return {"sm_mhz": statistics.median(s[0] for s in load), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "samples_under_load": len(load),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
+
+
+def config_of(w, world, nbytes):
+    """The workload description both arms print (identical keys, so the lines compare)."""
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len,
+            "len_range": list(w.len_range) if w.len_range else None, "h": w.h, "d_h": w.d_h,
+            "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
+            "reading": "summed" if w.summed else "partitioned", "l2": "inputs larger than L2",
+            "parallelism": f"replicas{world}", "cache_bytes_per_step": nbytes}
 
 
 def dist_setup(impl):
@@ -230,12 +283,15 @@ def oracle_sample_rate(w, inp, pairs_per_step, steps, warmup):
         step()
     # gathering rows is the oracle's page walk; it is timed too, per sequence first seen
     sub_pools.clear()
-    t0 = time.perf_counter()
+    t0, c0 = time.perf_counter(), time.process_time()
     for _ in range(steps):
         step()
-    dt = time.perf_counter() - t0
+    dt, cpu = time.perf_counter() - t0, time.process_time() - c0
     bytes_done = full_bytes * (pairs_per_step * steps) / total_heads
-    return bytes_done / dt / 1e9, dt / steps, threads
+    # threads the oracle actually kept busy: process CPU time over wall time (its BLAS pool may
+    # be larger, but one small matrix-vector product at a time leaves most of it idle)
+    cores = round(max(1.0, cpu / dt), 1)
+    return bytes_done / dt / 1e9, dt / steps, cores, threads
 
 
 def run_reference(args, world, rank):
@@ -244,19 +300,19 @@ def run_reference(args, world, rank):
     w = W.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.make_workload(w, device=dev)
-    rate, sec_per_step, threads = oracle_sample_rate(w, inp, 1, args.steps, args.warmup)
+    rate, sec_per_step, cores, pool_threads = oracle_sample_rate(w, inp, 1, args.steps, args.warmup)
+    nbytes = cache_bytes(w, inp["seq_lens"].cpu().tolist())
     line = {
         "impl": "reference",
         "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
-                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64,
-                   "reading": "summed" if w.summed else "partitioned"},
-        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "config": config_of(w, world, nbytes),
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "blas_pool_threads": pool_threads,
+                         "kind": "oracle",
                          "sample": "each step: the float64 oracle on one random (sequence, head) pair "
                                    f"of the {w.name} workload; value scaled by the fraction of the "
-                                   "workload's heads covered"},
+                                   "workload's heads covered; cores = process CPU time / wall time"},
         "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -266,6 +322,68 @@ def run_reference(args, world, rank):
 # our CUDA path
 # ---------------------------------------------------------------------------------------
 
+# the other benchmark configurations, timed in the same run as the headline (decode step and
+# kernels); each is a fresh workload on the device
+EXTRA_WORKLOADS = ["mlra2_h128_b64_n4096", "mlra4_h128_b8_n131072", "mlra4_h128_b128_ragged1k_32k",
+                   "mla_h128_b128_ragged1k_32k", "mlra4sum_h128_b32_n8192", "mlra2sum_h128_b64_n4096"]
+
+
+def make_handle(M, w, inp):
+    return M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed)
+
+
+def time_decode(M, w, inp, hdl, dev, steps, warmup):
+    """Whole-step time (CUDA events around `steps` back-to-back calls, kernels chained by
+    programmatic dependent launch) and per-kernel times (mlra_decode_profiled: events between
+    the kernels, no overlap), after a status-checked call and `warmup` untimed steps."""
+    out = torch.empty(w.batch, w.h, w.d_h, device=dev, dtype=torch.bfloat16)
+    ws = M.alloc_workspace(hdl, w.batch, dev)
+    stream = torch.cuda.current_stream(dev)
+    args_dec = (hdl, inp["q"], inp["pool"], inp["page_table"], inp["seq_lens"], out)
+    M.mlra_decode(*args_dec, workspace=ws)
+    torch.cuda.synchronize()
+    status = M.mlra_get_status(ws)
+    if status != 0:
+        raise RuntimeError(f"{w.name}: decode status {status}")
+    for _ in range(warmup):
+        M.mlra_decode(*args_dec, workspace=ws)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        M.mlra_decode(*args_dec, workspace=ws)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = ev0.elapsed_time(ev1) / steps
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        M.mlra_decode_profiled(*args_dec, kevs[i], workspace=ws)
+    torch.cuda.synchronize()
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kevs) / steps for i in range(3)]
+    return {"step_ms": step_ms, "k_ms": k_ms, "out": out, "ws": ws, "args": args_dec, "stream": stream}
+
+
+def roofline_of(w, seq_lens, decode_ms):
+    """Roofline of the decode kernel: HBM for the partitioned reading (below the ridge), the
+    bf16 tensor peak for the summed one (k times the MMA work per cached byte)."""
+    nbytes = cache_bytes(w, seq_lens)
+    peak, peak_kind = measured_hbm_peak()
+    tpeak, tpeak_kind = measured_bf16_peak()
+    achieved = nbytes / (decode_ms * 1e-3) / 1e9
+    flops = decode_flops(w, seq_lens)
+    tflops = flops / (decode_ms * 1e-3) / 1e12
+    if w.summed:
+        return {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s", "frac": tflops / tpeak,
+                "peak_kind": f"{tpeak_kind} dense bf16 (burst)", "flops_per_launch": flops,
+                "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak,
+                "kernel": "mlra_decode_kernel (split-KV latent attention, summed blocks)",
+                "traffic": recorded_traffic(w.name)}
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_kind": f"{peak_kind} copy bandwidth", "bytes_per_launch": nbytes,
+            "tensor_tflops": tflops, "tensor_frac": tflops / tpeak,
+            "kernel": "mlra_decode_kernel (split-KV latent attention)", "traffic": recorded_traffic(w.name)}
+
+
 def run_ours(args, world, rank, local):
     import rank_latent_kv_mlra_b200 as M
 
@@ -273,42 +391,17 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     w = W.WORKLOADS[args.workload]
     inp = W.make_workload(w, device=dev)
-    hdl = M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed)
+    hdl = make_handle(M, w, inp)
     B = w.batch
-    out = torch.empty(B, w.h, w.d_h, device=dev, dtype=torch.bfloat16)
-    ws = M.alloc_workspace(hdl, B, dev)
-    stream = torch.cuda.current_stream(dev)
-    args_dec = (hdl, inp["q"], inp["pool"], inp["page_table"], inp["seq_lens"], out)
-    nbytes = cache_bytes(w, inp["seq_lens"].cpu().tolist())
+    seq_lens = inp["seq_lens"].cpu().tolist()
+    nbytes = cache_bytes(w, seq_lens)
 
-    # correctness guard on this very launch configuration
-    M.mlra_decode(*args_dec, workspace=ws)
-    torch.cuda.synchronize()
-    status = M.mlra_get_status(ws)
-    if status != 0:
-        raise RuntimeError(f"decode status {status}")
-
-    for _ in range(args.warmup):
-        M.mlra_decode(*args_dec, workspace=ws)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        M.mlra_decode(*args_dec, workspace=ws)
-    ev1.record(stream)
-    torch.cuda.synchronize()
     barrier(world)
-    step_ms = ev0.elapsed_time(ev1) / args.steps
-
-    # per-kernel times: events between the three kernels (no programmatic overlap here)
-    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        M.mlra_decode_profiled(*args_dec, kevs[i], workspace=ws)
-    torch.cuda.synchronize()
-    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kevs) / args.steps for i in range(3)]
+    r = time_decode(M, w, inp, hdl, dev, args.steps, args.warmup)
+    barrier(world)
+    step_ms, k_ms, out, ws, stream = r["step_ms"], r["k_ms"], r["out"], r["ws"], r["stream"]
     clk = clocks.stop()
 
     # End to end through the public API: every step uploads its query and lengths from pinned
@@ -386,6 +479,30 @@ def run_ours(args, world, rank, local):
     # the pipelined steps computed the same output as the plain call
     assert torch.equal(out_host[(e2e_steps - 1) % NB], out.cpu())
 
+    # the other configurations, each timed the same way in this run
+    extra = {}
+    if not args.headline_only:
+        del inp, r
+        for name in EXTRA_WORKLOADS:
+            we = W.WORKLOADS[name]
+            ie = W.make_workload(we, device=dev)
+            he = make_handle(M, we, ie)
+            sl = ie["seq_lens"].cpu().tolist()
+            # about 0.2 s of timed steps per configuration, at least 20
+            n = max(20, min(args.steps, int(0.2e6 / max(1.0, cache_bytes(we, sl) / 4.0e6))))
+            re_ = time_decode(M, we, ie, he, dev, n, max(3, min(args.warmup, 20)))
+            st = max_over_ranks(re_["step_ms"], world, dev)
+            km = [max_over_ranks(x, world, dev) for x in re_["k_ms"]]
+            rf = roofline_of(we, sl, km[1])
+            extra[name] = {"steps": n, "step_us": st * 1e3, "decode_us": km[1] * 1e3,
+                           "absorb_us": km[0] * 1e3, "combine_uproj_us": km[2] * 1e3,
+                           "cache_bytes_per_step": cache_bytes(we, sl),
+                           "step_gbs": cache_bytes(we, sl) / (st * 1e-3) / 1e9,
+                           "roofline": {k2: rf[k2] for k2 in ("bound", "achieved", "peak", "unit", "frac")},
+                           "hbm_frac": rf.get("hbm_frac", rf["frac"])}
+            del ie, re_, he
+            torch.cuda.empty_cache()
+
     step_ms_max = max_over_ranks(step_ms, world, dev)
     e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
     k_ms = [max_over_ranks(x, world, dev) for x in k_ms]
@@ -394,34 +511,14 @@ def run_ours(args, world, rank, local):
 
     peak, peak_kind = measured_hbm_peak()
     value = world * nbytes / (step_ms_max * 1e-3) / 1e9
-    achieved = nbytes / (k_ms[1] * 1e-3) / 1e9
-    flops = decode_flops(w, inp["seq_lens"].cpu().tolist())
-    tflops = flops / (k_ms[1] * 1e-3) / 1e12
-    tpeak, tpeak_kind = measured_bf16_peak()
-    if w.summed:
-        # every block serves all h heads: k times the MMA work per cached byte, above the ridge
-        roofline = {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": tflops / tpeak, "peak_kind": f"{tpeak_kind} dense bf16 (burst)",
-                    "flops_per_launch": flops, "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak,
-                    "kernel": "mlra_decode_kernel (split-KV latent attention, summed blocks)",
-                    "traffic": recorded_traffic(w.name)}
-    else:
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
-                    "tensor_tflops": tflops, "tensor_frac": tflops / tpeak,
-                    "kernel": "mlra_decode_kernel (split-KV latent attention)",
-                    "traffic": recorded_traffic(w.name)}
+    roofline = roofline_of(w, seq_lens, k_ms[1])
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms_max, "us_per_step": step_ms_max * 1e3,
         "pct_of_hbm_peak": 100.0 * value / world / peak,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": f"synthetic (seeded; inputs larger than L2: the {nbytes / 1e6:.0f} MB cache stream evicts the 126 MB L2 each step)",
-        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "h": w.h, "d_h": w.d_h,
-                   "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
-                   "reading": "summed" if w.summed else "partitioned",
-                   "l2": "inputs larger than L2", "parallelism": f"replicas{world}",
-                   "cache_bytes_per_step": nbytes},
+        "config": config_of(w, world, nbytes),
         "kernels_ms": {"absorb": k_ms[0], "decode": k_ms[1], "combine_uproj": k_ms[2]},
         "roofline": roofline,
         "e2e": {"value": world * nbytes / (e2e_ms_max * 1e-3) / 1e9, "unit": UNIT,
@@ -433,15 +530,26 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
+    if clk and clk.get("sm_mhz"):
+        # step time scaled to the maximum SM clock: how the number would move with the clock
+        line["us_x_mhz"] = step_ms_max * 1e3 * clk["sm_mhz"]
+    if extra:
+        line["workloads"] = extra
     if world == 1 and not args.no_cpu_baseline:
         # a summed-blocks head attends to all k blocks: k times the oracle work per pair
         pairs = max(1, args.cpu_pairs // (w.k if w.summed else 1))
-        rate, sec, threads = oracle_sample_rate(w, inp, pairs, 1, 0)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+        rate, sec, cores, pool_threads = oracle_sample_rate(w, inp_for_cpu(w, dev), pairs, 1, 0)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "blas_pool_threads": pool_threads,
+                                "kind": "oracle",
                                 "sample": f"float64 oracle on {pairs} random (sequence, head) pairs of "
                                           f"{w.name} ({sec:.1f} s), scaled by the fraction of the "
-                                          "workload's heads covered"}
+                                          "workload's heads covered; cores = process CPU time / wall time"}
     print(json.dumps(line), flush=True)
+
+
+def inp_for_cpu(w, dev):
+    """The headline workload again (same seed, same values) for the CPU baseline."""
+    return W.make_workload(w, device=dev)
 
 
 def producer_bytes(w, batch, d_model):
@@ -478,7 +586,7 @@ def run_producer(args, world, rank, local):
         call()
     barrier(world)
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     stream = torch.cuda.current_stream(dev)
@@ -520,6 +628,8 @@ def main():
     ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
     ap.add_argument("--cpu-pairs", type=int, default=15000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip timing the other configurations (the `workloads` key)")
     ap.add_argument("--producer", action="store_true",
                     help="time the step before decoding (the new cache rows) instead of the decode step")
     args = ap.parse_args()
