@@ -39,10 +39,11 @@ FALLBACK_HBM_GBS = 6650.0
 
 def cache_bytes(w: W.Workload, seq_lens) -> int:
     """Algorithmic bytes of the latent-cache stream of one step: each cached token's row
-    [c | k^R] read once (bf16) plus one 4-byte page-table entry per 64 tokens."""
+    [c | k^R] read once (2 bytes per element in bf16, 1 in E4M3) plus one 4-byte page-table
+    entry per 64 tokens."""
     toks = int(sum(int(n) for n in seq_lens))
     pages = int(sum((int(n) + 63) // 64 for n in seq_lens))
-    return toks * (w.d_c + w.d_r) * 2 + pages * 4
+    return toks * (w.d_c + w.d_r) * (1 if w.cache == "e4m3" else 2) + pages * 4
 
 
 def measured_hbm_peak():
@@ -122,14 +123,18 @@ class ClockSampler:
         self.smi = None
 
     def _nvml_handle(self):
+        """The NVML handle of this process's CUDA device, matched by UUID (NVML enumerates
+        every GPU of the machine, whatever CUDA_VISIBLE_DEVICES hides)."""
         import pynvml
         pynvml.nvmlInit()
-        bus = torch.cuda.get_device_properties(self.device).pci_bus_id  # e.g. 0000:1B:00.0
-        try:
-            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-        except Exception:
-            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
-        return pynvml, h
+        want = str(torch.cuda.get_device_properties(self.device).uuid).lower().replace("gpu-", "")
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = (u.decode() if isinstance(u, bytes) else str(u)).lower().replace("gpu-", "")
+            if u == want:
+                return pynvml, h
+        raise RuntimeError("no NVML device with this CUDA device's UUID")
 
     def start(self):
         import threading
@@ -209,7 +214,7 @@ def config_of(w, world, nbytes):
     return {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len,
             "len_range": list(w.len_range) if w.len_range else None, "h": w.h, "d_h": w.d_h,
             "d_c": w.d_c, "d_r": w.d_r, "k": w.k, "page_size": 64, "paging": w.paging,
-            "reading": "summed" if w.summed else "partitioned", "l2": "inputs larger than L2",
+            "reading": "summed" if w.summed else "partitioned", "cache": w.cache, "l2": "inputs larger than L2",
             "parallelism": f"replicas{world}", "cache_bytes_per_step": nbytes}
 
 
@@ -266,7 +271,12 @@ def oracle_sample_rate(w, inp, pairs_per_step, steps, warmup):
         if b not in sub_pools:
             n = int(seq_lens[b])
             pages = pt[b, :(n + 63) // 64]
-            sp = inp["pool"][torch.as_tensor(pages, device=inp["pool"].device).long()].float().cpu().numpy()
+            sp = inp["pool"][torch.as_tensor(pages, device=inp["pool"].device).long()]
+            if w.cache == "e4m3":
+                from oracle import fp8_cache_oracle as F
+                sp = F.dequantize_pool(sp.cpu().numpy(), w.d_c, W.E4M3_SCALE, W.E4M3_SCALE)
+            else:
+                sp = sp.float().cpu().numpy()
             sub_pools[b] = O.gather_rows(sp, np.arange(len(pages))[None, :], 0, n)
         return sub_pools[b]
 
@@ -325,11 +335,13 @@ def run_reference(args, world, rank):
 # the other benchmark configurations, timed in the same run as the headline (decode step and
 # kernels); each is a fresh workload on the device
 EXTRA_WORKLOADS = ["mlra2_h128_b64_n4096", "mlra4_h128_b8_n131072", "mlra4_h128_b128_ragged1k_32k",
-                   "mla_h128_b128_ragged1k_32k", "mlra4sum_h128_b32_n8192", "mlra2sum_h128_b64_n4096"]
+                   "mla_h128_b128_ragged1k_32k", "mlra4sum_h128_b32_n8192", "mlra2sum_h128_b64_n4096",
+                   "mlra4fp8_h128_b32_n8192"]
 
 
 def make_handle(M, w, inp):
-    return M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed)
+    fp8 = dict(cache_fp8=True, latent_scale=W.E4M3_SCALE, rope_scale=W.E4M3_SCALE) if w.cache == "e4m3" else {}
+    return M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inp["w_uk"], inp["w_uv"], blocks_summed=w.summed, **fp8)
 
 
 def time_decode(M, w, inp, hdl, dev, steps, warmup):
@@ -494,7 +506,7 @@ def run_ours(args, world, rank, local):
             st = max_over_ranks(re_["step_ms"], world, dev)
             km = [max_over_ranks(x, world, dev) for x in re_["k_ms"]]
             rf = roofline_of(we, sl, km[1])
-            extra[name] = {"steps": n, "step_us": st * 1e3, "decode_us": km[1] * 1e3,
+            extra[name] = {"cache": we.cache, "steps": n, "step_us": st * 1e3, "decode_us": km[1] * 1e3,
                            "absorb_us": km[0] * 1e3, "combine_uproj_us": km[2] * 1e3,
                            "cache_bytes_per_step": cache_bytes(we, sl),
                            "step_gbs": cache_bytes(we, sl) / (st * 1e-3) / 1e9,

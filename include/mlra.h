@@ -79,6 +79,14 @@ typedef struct {
   float attn_scale;    /* alpha_attn when blocks_summed: <= 0 selects 1/sqrt(k), the values the
                           MLRA index page's appendix model tables print for MLRA-2 (sqrt(2)/2)
                           and MLRA-4 (1/2). Ignored otherwise. */
+  int cache_fp8;       /* 0: bf16 cache. 1: E4M3 cache (the lesty.tech MLA article, section 5:
+                          FP8 storage of the cached latent): every element of a cached row
+                          [c | k^R] is one OCP E4M3 byte; the pool is then uint8
+                          [num_pages][page_size][d_c + d_rope]. */
+  float latent_scale;  /* E4M3 cache: value of a latent byte = latent_scale * e4m3(byte);
+                          <= 0 selects 1. Ignored for a bf16 cache. */
+  float rope_scale;    /* E4M3 cache: value of a RoPE-key byte = rope_scale * e4m3(byte);
+                          <= 0 selects 1. Ignored for a bf16 cache. */
 } mlra_config;
 
 /* Compiled dims (others return MLRA_ERR_UNSUPPORTED), as (d_c/k, d_rope, heads per block, d_h),
@@ -86,7 +94,7 @@ typedef struct {
  *   (32, 16, <=16, 32), (128, 64, <=32 or a multiple of 32, 128),
  *   (256, 64, <=64 or a multiple of 64, 128), (512, 64, <=64 or a multiple of 64, 128);
  * blocks_summed with k = 4 and (32, 16, ...) or (128, 64, ...), or k = 2 and (256, 64, ...);
- * batch <= 4096. */
+ * cache_fp8 with (128, 64, a multiple of 32, 128) and blocks_summed = 0; batch <= 4096. */
 
 typedef struct mlra_ctx* mlra_handle;
 
@@ -106,7 +114,8 @@ int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes);
 /* One decode step for `batch` sequences.
  *   q          device [batch][h][d_h + d_rope], q^C_h then q^R_h (already rotated),
  *              dtype q_dtype (F32 or BF16; converted to bf16 for the tensor cores).
- *   pool       device bf16 [num_pages][page_size][d_c + d_rope]: token row = [c_1..c_k | k^R].
+ *   pool       device bf16 [num_pages][page_size][d_c + d_rope]: token row = [c_1..c_k | k^R]
+ *              (uint8 E4M3 bytes of the same shape when the handle has cache_fp8).
  *              16-byte aligned. Slots past a sequence's length may hold anything.
  *   page_table device int32 [batch][pt_stride]: token t of sequence b lives in slot
  *              t % page_size of page page_table[b*pt_stride + t/page_size].
@@ -175,7 +184,10 @@ int mlra_decode_profiled(mlra_handle h, const void* q, mlra_dtype q_dtype, const
 /* Writes new cache rows: token i goes to sequence seq_ids[i] at position positions[i], i.e.
  * slot positions[i] % page_size of page page_table[seq_ids[i]*pt_stride + positions[i]/page_size].
  *   c_new   device [n_tokens][d_c], kr_new device [n_tokens][d_rope], dtype in_dtype;
- *           F32 input is rounded to bf16 to nearest-even.
+ *           F32 input is rounded to bf16 to nearest-even. With an E4M3 cache (cache_fp8) each
+ *           element v is stored as the E4M3 byte nearest to v / scale (the quotient in fp32;
+ *           ties to even; saturated at +-448), scale being latent_scale for c_new and
+ *           rope_scale for kr_new.
  *   page_table has `batch` rows of pt_stride entries; seq_ids[i] must be < batch.
  *   status  device int32 word that receives a device error code (first error wins), or NULL.
  * Rows whose page id falls outside [0, num_pages), or whose sequence / position falls outside
@@ -199,7 +211,8 @@ int mlra_project_workspace_size(mlra_handle h, int batch, int d_model, size_t* b
  *                           pos * rope_base^(-2i/d_rope), RoFormer's rotation, which the pages
  *                           cite but do not spell out)
  * and writes the bf16 (round to nearest even) row [c | k^R] into slot pos % page_size of page
- * page_table[b*pt_stride + pos/page_size].
+ * page_table[b*pt_stride + pos/page_size]; with an E4M3 cache, the bytes e4m3(v / scale) as in
+ * mlra_append_cache.
  *   x          device bf16 [batch][d_model], 16-byte aligned; d_model a multiple of 128.
  *   w_down     device bf16 [d_c + d_rope][d_model], 16-byte aligned: row r holds the weights
  *              of output feature r (the d_c latent features, then the d_rope RoPE-key

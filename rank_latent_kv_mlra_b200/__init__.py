@@ -30,6 +30,7 @@ STATUS = {
     -6: "MLRA_ERR_WORKSPACE",
     -7: "MLRA_ERR_SEQ_LEN",
     -8: "MLRA_ERR_SCRATCH_LIMIT",
+    -9: "MLRA_ERR_DRAIN",
 }
 
 EXPORTED = [
@@ -49,7 +50,8 @@ class mlra_config(ctypes.Structure):
     _fields_ = [("h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_c", ctypes.c_int),
                 ("d_rope", ctypes.c_int), ("k", ctypes.c_int), ("page_size", ctypes.c_int),
                 ("softmax_scale", ctypes.c_float), ("blocks_summed", ctypes.c_int),
-                ("attn_scale", ctypes.c_float)]
+                ("attn_scale", ctypes.c_float), ("cache_fp8", ctypes.c_int),
+                ("latent_scale", ctypes.c_float), ("rope_scale", ctypes.c_float)]
 
 
 class mlra_info(ctypes.Structure):
@@ -140,16 +142,20 @@ class Handle:
 
 def mlra_create(h: int, d_h: int, d_c: int, d_rope: int, k: int, w_uk: torch.Tensor,
                 w_uv: torch.Tensor, softmax_scale: float = 0.0, page_size: int = 64,
-                blocks_summed: bool = False, attn_scale: float = 0.0) -> Handle:
+                blocks_summed: bool = False, attn_scale: float = 0.0, cache_fp8: bool = False,
+                latent_scale: float = 1.0, rope_scale: float = 1.0) -> Handle:
     """blocks_summed: every head attends to every block with weights [k][h][d_c/k][d_h] and the
-    per-block outputs are summed times attn_scale (<= 0: 1/sqrt(k)); lse is then [batch][k*h]."""
+    per-block outputs are summed times attn_scale (<= 0: 1/sqrt(k)); lse is then [batch][k*h].
+    cache_fp8: the pool holds E4M3 bytes (uint8), a latent byte e meaning latent_scale *
+    e4m3(e) and a RoPE-key byte rope_scale * e4m3(e)."""
     lib = load_library()
     shape = (k, h, d_c // k, d_h) if blocks_summed else (h, d_c // k, d_h)
     for t, n in ((w_uk, "w_uk"), (w_uv, "w_uv")):
         _require(t, n, torch.bfloat16)
         if tuple(t.shape) != shape:
             raise ValueError(f"{n} must be {'[k][h]' if blocks_summed else '[h]'}[d_c/k][d_h]")
-    cfg = mlra_config(h, d_h, d_c, d_rope, k, page_size, softmax_scale, int(blocks_summed), attn_scale)
+    cfg = mlra_config(h, d_h, d_c, d_rope, k, page_size, softmax_scale, int(blocks_summed), attn_scale,
+                      int(cache_fp8), latent_scale, rope_scale)
     out = ctypes.c_void_p()
     _check(lib.mlra_create(ctypes.byref(cfg), _ptr(w_uk), _ptr(w_uv), ctypes.byref(out)), "mlra_create")
     return Handle(out, cfg, w_uk, w_uv)
@@ -172,9 +178,13 @@ def mlra_get_info(handle: Handle) -> dict:
     return {f: getattr(info, f) for f, _ in mlra_info._fields_}
 
 
+def _pool_dtype(handle):
+    return torch.uint8 if handle.cfg.cache_fp8 else torch.bfloat16
+
+
 def _decode_common(handle, q, pool, page_table, seq_lens, workspace):
     _require(q, "q")
-    _require(pool, "pool", torch.bfloat16)
+    _require(pool, "pool", _pool_dtype(handle))
     _require(page_table, "page_table", torch.int32)
     _require(seq_lens, "seq_lens", torch.int32)
     _require(workspace, "workspace")
@@ -213,7 +223,7 @@ def mlra_decode_noalloc(handle: Handle, q, pool, page_table, seq_lens, out, lse=
     that receives the call's device status. Raises MlraError(MLRA_ERR_SCRATCH_LIMIT) for a
     batch the array cannot hold."""
     _require(q, "q")
-    _require(pool, "pool", torch.bfloat16)
+    _require(pool, "pool", _pool_dtype(handle))
     _require(page_table, "page_table", torch.int32)
     _require(seq_lens, "seq_lens", torch.int32)
     _require(out, "out")
@@ -270,7 +280,7 @@ def mlra_decode_latent(handle: Handle, q, pool, page_table, seq_lens, latent_out
 
 def mlra_append_cache(handle: Handle, pool, page_table, seq_ids, positions, c_new, kr_new,
                       status=None, stream=None):
-    _require(pool, "pool", torch.bfloat16)
+    _require(pool, "pool", _pool_dtype(handle))
     for t, n in ((page_table, "page_table"), (seq_ids, "seq_ids"), (positions, "positions")):
         _require(t, n, torch.int32)
     _require(c_new, "c_new")
@@ -298,7 +308,7 @@ def mlra_project_append(handle: Handle, x, w_down, positions, pool, page_table, 
     _require(x, "x", torch.bfloat16)
     _require(w_down, "w_down", torch.bfloat16)
     _require(positions, "positions", torch.int32)
-    _require(pool, "pool", torch.bfloat16)
+    _require(pool, "pool", _pool_dtype(handle))
     _require(page_table, "page_table", torch.int32)
     cfg = handle.cfg
     B, d_model = x.shape

@@ -43,6 +43,46 @@ __global__ void mlra_append_kernel(__nv_bfloat16* __restrict__ pool, int num_pag
   }
 }
 
+// E4M3 cache: one warp per new token writes the bytes e4m3(v / scale) of its row (v / scale in
+// fp32, then rounded to the nearest E4M3 value, ties to even, saturated at +-448); the latent
+// columns use latent_scale, the RoPE columns rope_scale.
+__global__ void mlra_append_e4m3_kernel(uint8_t* __restrict__ pool, int num_pages,
+                                        const int* __restrict__ page_table, int pt_stride, int batch,
+                                        const int* __restrict__ seq_ids, const int* __restrict__ positions,
+                                        const void* c_new, const void* kr_new, int in_f32, int n_tokens,
+                                        int d_c, int d_r, float latent_scale, float rope_scale, int* status) {
+  const int i = blockIdx.x * (blockDim.x / 32) + warp_id();
+  const int lane = lane_id();
+  if (i >= n_tokens) return;
+  const int b = __ldg(seq_ids + i), pos = __ldg(positions + i);
+  if (b < 0 || b >= batch || pos < 0 || pos / kPage >= pt_stride) {
+    if (lane == 0) set_status(status, kErrSeqLen);
+    return;
+  }
+  const int page = __ldg(page_table + (size_t)b * pt_stride + pos / kPage);
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) set_status(status, kErrPageOob);
+    return;
+  }
+  const int D = d_c + d_r;
+  uint8_t* row = pool + ((size_t)page * kPage + pos % kPage) * D;
+  for (int e = lane; e < D; e += 32) {
+    float v;
+    if (e < d_c) {
+      const size_t s = (size_t)i * d_c + e;
+      v = in_f32 ? __ldg(static_cast<const float*>(c_new) + s)
+                 : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(c_new) + s));
+      v = __fdiv_rn(v, latent_scale);
+    } else {
+      const size_t s = (size_t)i * d_r + (e - d_c);
+      v = in_f32 ? __ldg(static_cast<const float*>(kr_new) + s)
+                 : __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(kr_new) + s));
+      v = __fdiv_rn(v, rope_scale);
+    }
+    row[e] = static_cast<uint8_t>(e4m3x2_from_f32(v, 0.f) & 0xFF);
+  }
+}
+
 // Single CTA: writes every segment (b, group, tile_begin, tile_end, slot) of the plan in
 // group order, using the same device routines as the decode and combine kernels.
 __global__ void __launch_bounds__(192, 1)

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -264,6 +265,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D(tmem) (+)= A(smem desc) * B(smem desc), E4M3 inputs (K = 32 per instruction), fp32
+// accumulate. One thread issues.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrives on `bar` once every tcgen05 MMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -418,6 +430,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0) and an fp32
+// accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Byte offset of logical byte `off` inside a swizzled region whose rows are `row_bytes`
 // wide (the pattern the TMA engine writes and the tensor core reads): the 16-byte chunk
 // index bits [4, 4+b) are XORed with address bits [7, 7+b), b = log2(row_bytes / 16).
@@ -429,6 +448,42 @@ __device__ __forceinline__ uint32_t swizzle(uint32_t off, int row_bytes) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// E4M3 conversions (round to nearest even, saturating at +-448). The first argument of the
+// two-element forms lands in the lower byte, i.e. first in memory.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint16_t e4m3x2_from_f16x2(uint32_t h2) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h2));
+  return r;
+}
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t e2) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(e2));
+  return r;
+}
+__device__ __forceinline__ uint32_t f16x2_from_f32(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Two non-negative values as a pair of E4M3 terms each, value ~= hi + lo: hi is the nearest
+// E4M3 value, lo the nearest to the remainder (about 7 significant bits in all). The split
+// goes through f16 (exact for every E4M3 value; 11 bits for the input).
+__device__ __forceinline__ void e4m3x2_split(float a, float b, uint16_t& hi, uint16_t& lo) {
+  const uint32_t v = f16x2_from_f32(a, b);
+  hi = e4m3x2_from_f16x2(v);
+  lo = e4m3x2_from_f16x2(sub_f16x2(v, f16x2_from_e4m3x2(hi)));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

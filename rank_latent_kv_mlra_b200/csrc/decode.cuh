@@ -22,9 +22,9 @@
 // barriers. The roles hand off through mbarriers; each wait is bounded (see mbar_wait).
 //
 // Softmax detail: each thread owns one token row of S^T and all its heads. The running
-// maximum m_h is only raised when some score exceeds it by more than kRescaleSlack (in
-// log2 units); otherwise P = exp2(s - m_h) is used as is (values up to 2^slack are exact in
-// fp32/bf16 range). A raise costs a cross-thread max and a rescale of O in TMEM; it happens
+// maximum m_h is only raised when some score exceeds it by more than the shape's SLACK (in
+// log2 units); otherwise P = exp2(s - m_h) is used as is (values up to 2^slack stay inside
+// the range of P's storage type). A raise costs a cross-thread max and a rescale of O in TMEM; it happens
 // on a segment's first tile and then rarely.
 #pragma once
 
@@ -32,16 +32,27 @@
 
 namespace mlra {
 
-constexpr float kRescaleSlack = 8.0f;
 constexpr int kPlanBar = 5;  // named barrier of the segment-list hand-off (1..4: softmax groups)
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2>
+template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2, bool FP8_ = false>
 struct DecodeShape {
   static constexpr int DB = DB_;      // latent block width d_c / k
   static constexpr int DR = DR_;      // RoPE key width
-  static constexpr int NP = NP_;      // heads per CTA (MMA N), 16 / 32 / 64
+  static constexpr int NP = NP_;      // heads per CTA, 16 / 32 / 64
+  // E4M3 cache: every cached element is one byte, and the MMAs run on E4M3 operands. The query
+  // and P are then each carried as two E4M3 terms (hi + lo) in two column sets of N, so N = 2 NP
+  // (an MMA costs the same up to N = 128).
+  static constexpr bool FP8 = FP8_;
+  static constexpr int EB = FP8 ? 1 : 2;   // bytes per cached element
+  static constexpr int NQ = FP8 ? 2 : 1;   // query / P terms per head
+  static constexpr int MN = NQ * NP;       // MMA N
+  static constexpr int KT = 32 / EB;       // tokens per PV K step (32 bytes of K per MMA)
+  // P is written as p * P_SCALE (E4M3 split), with the lazy maximum's slack lowered so that
+  // p * P_SCALE <= 2^(SLACK + log2 P_SCALE) = 256 stays inside E4M3's range
+  static constexpr float SLACK = FP8 ? 3.0f : 8.0f;
+  static constexpr float P_SCALE = FP8 ? 32.0f : 1.0f;
   static constexpr int NWG = 2;       // softmax warpgroups; each owns NP / NWG heads
   static constexpr int HW = NP / NWG;
   static constexpr int PV_WARP = 2 + 4 * NWG;  // after the softmax warps
@@ -58,21 +69,22 @@ struct DecodeShape {
   // before the phase it held has been waited for (no parity aliasing), however far the softmax
   // runs ahead of the PV issuer.
   static constexpr int PR = STAGES > 2 ? STAGES : 2;
-  // A cache row is split into swizzle-width regions: block columns and RoPE columns.
-  static constexpr int CW = DB < 64 ? DB : 64;
+  // A cache row is split into swizzle-width regions (at most 128 bytes): block columns and RoPE
+  // columns.
+  static constexpr int CW = DB * EB < 128 ? DB : 128 / EB;
   static constexpr int NC = DB / CW;
-  static constexpr int RW = DR < 64 ? DR : 64;
+  static constexpr int RW = DR * EB < 128 ? DR : 128 / EB;
   static constexpr int NR = DR / RW;
-  static constexpr int C_ROWB = CW * 2;
-  static constexpr int R_ROWB = RW * 2;
+  static constexpr int C_ROWB = CW * EB;
+  static constexpr int R_ROWB = RW * EB;
   static constexpr int C_REG = round_up(kTile * C_ROWB, 1024);
   static constexpr int R_REG = round_up(kTile * R_ROWB, 1024);
   static constexpr int STAGE_BYTES = NC * C_REG + NR * R_REG;
   static constexpr int PAGE_TX = NC * kPage * C_ROWB + NR * kPage * R_ROWB;
-  static constexpr int QC_REG = round_up(NP * C_ROWB, 1024);
-  static constexpr int QR_REG = round_up(NP * R_ROWB, 1024);
+  static constexpr int QC_REG = round_up(MN * C_ROWB, 1024);
+  static constexpr int QR_REG = round_up(MN * R_ROWB, 1024);
   static constexpr int Q_BYTES = NC * QC_REG + NR * QR_REG;
-  static constexpr int P_ROWB = NP * 2;
+  static constexpr int P_ROWB = NP * 2;  // NP bf16, or NQ * NP E4M3 bytes
   static constexpr int P_BYTES = round_up(kTile * P_ROWB, 1024);
   static constexpr int NMT = DB >= 128 ? DB / 128 : 1;  // PV M tiles
   // A stage is loaded and freed in NG groups, one per PV M tile (128 latent features); the RoPE
@@ -80,12 +92,12 @@ struct DecodeShape {
   // the PV MMAs of its M tile have read it, so with several M tiles (d_b = 256, 512) the next
   // tile's first columns stream in while this tile's PV is still running.
   static constexpr int NG = NMT;
-  static constexpr int RPG = (DB / (DB < 64 ? DB : 64)) / NMT;  // block regions per group
+  static constexpr int RPG = NC / NMT;  // block regions per group
   static constexpr uint32_t PV_LBO = DB >= 128 ? C_REG : 0;  // next 64-feature chunk
-  static constexpr int SBUF = SBUF_;                // S buffers of NP columns in TMEM
+  static constexpr int SBUF = SBUF_;                // S buffers of MN columns in TMEM
   static constexpr int S_COL0 = 0;
-  static constexpr int O_COL = SBUF * NP;           // NMT x NP columns
-  static constexpr int TMEM_USED = SBUF * NP + NMT * NP;
+  static constexpr int O_COL = SBUF * MN;           // NMT x MN columns
+  static constexpr int TMEM_USED = SBUF * MN + NMT * MN;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int MAX_SEGS = 64;
@@ -108,6 +120,7 @@ struct DecodeShape {
   static constexpr int SMEM_BYTES = OFF_MISC + 64 * 4 + 1024;  // + alignment slack
   static_assert(DB % CW == 0 && DR % RW == 0, "region split");
   static_assert(NP == 16 || NP == 32 || NP == 64, "heads per CTA");
+  static_assert(!FP8 || (NMT == 1 && MN <= 128 && R_ROWB == 64), "E4M3 shapes: one PV M tile, 64-byte RoPE rows");
   static_assert(QBUF == 1 || QBUF == 2, "query buffers");
   static_assert(SBUF >= 2 && TMEM_USED <= 512, "S buffers");
   static_assert(SMEM_BYTES <= 227 * 1024, "dynamic shared memory of one sm_100 CTA");
@@ -129,6 +142,8 @@ struct DecodeParams {
   int h;            // total heads
   int d_c;          // column of k^R in a cache row
   int q_rows;       // query rows a CTA loads: min(h/k, NP); rows past them stay zero
+  const float* qfac;  // E4M3 cache: [batch][nsub][NP] factor of each head's query terms
+  float o_scale;    // E4M3 cache: latent scale / P scale, applied to the partial outputs
   float* o_part;    // [slots][h][DB] fp32, normalised partial latent outputs
   float* lse_part;  // [slots][h] fp32, log2-domain log-sum-exp
   int* status;
@@ -204,6 +219,15 @@ __device__ __forceinline__ void add_f32x2(float& d0, float& d1, float a0, float 
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2pack(a0, a1)), "l"(f2pack(b0, b1)));
   d0 = __uint_as_float(static_cast<uint32_t>(d));
   d1 = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+
+// One MMA of the shape's kind: bf16 (K = 16) or E4M3 (K = 32).
+template <class Sh>
+__device__ __forceinline__ void shape_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (Sh::FP8)
+    umma_e4m3(d, a, b, idesc, acc);
+  else
+    umma_bf16(d, a, b, idesc, acc);
 }
 
 template <class Sh>
@@ -390,8 +414,8 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           ok = mbar_wait(&qempty_bar[qb], ((segc / Sh::QBUF) & 1) ^ 1, abort_flag, p.wait_limit_ns);
           if (ok) {
             uint8_t* qdst = qbufs + qb * Sh::Q_BYTES;
-            mbar_arrive_expect_tx(&qfull_bar[qb], p.q_rows * (Sh::DB + Sh::DR) * 2);
-            const int qrow = (sg.b * p.nsub + sub) * NP;
+            mbar_arrive_expect_tx(&qfull_bar[qb], Sh::NQ * p.q_rows * (Sh::DB + Sh::DR) * Sh::EB);
+            const int qrow = (sg.b * p.nsub + sub) * Sh::MN;
             for (int r = 0; r < Sh::NC; ++r)
               tma_load_2d(qdst + r * Sh::QC_REG, &map_qc, &qfull_bar[qb], r * Sh::CW, qrow, pol_keep);
             for (int r = 0; r < Sh::NR; ++r)
@@ -465,7 +489,8 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       // contents. The PVs have their own issuing warp, so a finished P never waits behind a
       // QK wait here.
       if (lane == 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NP, false, false);
+        constexpr uint32_t idesc_qk = Sh::FP8 ? idesc_e4m3_f32(128, Sh::MN, false, false)
+                                              : idesc_bf16_f32(128, NP, false, false);
         uint32_t ci = it, sc = segc;
         bool ok = true;
         for (int si = 0; si < nseg && ok; ++si) {
@@ -478,7 +503,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             MLRA_TRACE_POINT(1, 432 + min((int)ci, 31));
             const uint32_t st_addr = smem_u32(stages + (ci % STAGES) * Sh::STAGE_BYTES);
             const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
-            const uint32_t d = tbase + Sh::S_COL0 + (ci % Sh::SBUF) * NP;
+            const uint32_t d = tbase + Sh::S_COL0 + (ci % Sh::SBUF) * Sh::MN;
             uint32_t acc = 0;
             // each column group's MMAs go out as soon as that group has landed
 #pragma unroll
@@ -495,7 +520,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                                                swizzle_code(Sh::C_ROWB));
                   const uint64_t b = smem_desc(q_addr + r * Sh::QC_REG + ks * 32, 16, 8 * Sh::C_ROWB,
                                                swizzle_code(Sh::C_ROWB));
-                  umma_bf16(d, a, b, idesc_qk, acc);
+                  shape_mma<Sh>(d, a, b, idesc_qk, acc);
                   acc = 1;
                 }
               }
@@ -508,7 +533,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                                                  8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
                     const uint64_t b = smem_desc(q_addr + Sh::NC * Sh::QC_REG + r * Sh::QR_REG + ks * 32, 16,
                                                  8 * Sh::R_ROWB, swizzle_code(Sh::R_ROWB));
-                    umma_bf16(d, a, b, idesc_qk, 1);
+                    shape_mma<Sh>(d, a, b, idesc_qk, 1);
                   }
                 }
               }
@@ -532,7 +557,8 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       // One thread issues O^T += C_j^T(i) P^T(i) as soon as both softmax warpgroups have
       // written P(i), then frees tile i's pipeline stage and signals pvdone.
       if (lane == 0) {
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NP, true, true);
+        constexpr uint32_t idesc_pv = Sh::FP8 ? idesc_e4m3_f32(128, Sh::MN, true, true)
+                                              : idesc_bf16_f32(128, NP, true, true);
         uint32_t pi = it;
         bool ok = true;
         for (int si = 0; si < nseg && ok; ++si) {
@@ -550,12 +576,12 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
 #pragma unroll
-              for (int ks = 0; ks < kTile / 16; ++ks) {
-                const uint64_t a = smem_desc(st_addr + mt * (128 / Sh::CW) * Sh::C_REG + ks * 16 * Sh::C_ROWB,
+              for (int ks = 0; ks < kTile / Sh::KT; ++ks) {
+                const uint64_t a = smem_desc(st_addr + mt * (128 / Sh::CW) * Sh::C_REG + ks * Sh::KT * Sh::C_ROWB,
                                              Sh::PV_LBO, 8 * Sh::C_ROWB, swizzle_code(Sh::C_ROWB));
-                const uint64_t b = smem_desc(p_addr + ks * 16 * Sh::P_ROWB, Sh::P_BYTES, 8 * Sh::P_ROWB,
+                const uint64_t b = smem_desc(p_addr + ks * Sh::KT * Sh::P_ROWB, Sh::P_BYTES, 8 * Sh::P_ROWB,
                                              swizzle_code(Sh::P_ROWB));
-                umma_bf16(tbase + Sh::O_COL + mt * NP, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
+                shape_mma<Sh>(tbase + Sh::O_COL + mt * Sh::MN, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
               }
               // this M tile's columns are read: its group may be reloaded (the last group also
               // holds the RoPE columns and P, read by every M tile)
@@ -588,10 +614,22 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       float m_reg[Sh::M_SMEM ? 1 : HW];
       float* m_sm = reinterpret_cast<float*>(smem + Sh::OFF_M) + (warp - 2) * HW;
       auto m = [&](int x) -> float& { return Sh::M_SMEM ? m_sm[x] : m_reg[x % (Sh::M_SMEM ? 1 : HW)]; };
+      // E4M3 cache: each head's query terms carry a power-of-two factor (absorb kernel), read
+      // from the workspace once per segment; the absorb kernel must have finished writing it
+      float qf[Sh::FP8 ? HW : 1];
+      if constexpr (Sh::FP8) grid_dependency_wait();
       bool ok = true;
       for (int si = 0; si < nseg && ok; ++si) {
         const Segment sg = segs[si];
         const int slot = sg.b + group;
+        if constexpr (Sh::FP8) {
+          const float4* fsrc = reinterpret_cast<const float4*>(p.qfac + ((size_t)sg.b * p.nsub + sub) * NP + hcol);
+#pragma unroll
+          for (int x = 0; x < HW; x += 4) {
+            const float4 f = __ldg(fsrc + x / 4);
+            qf[x] = f.x; qf[x + 1] = f.y; qf[x + 2] = f.z; qf[x + 3] = f.w;
+          }
+        }
         for (int t = sg.tile_begin; t < sg.tile_end; ++t, ++it) {
           const bool first = (t == sg.tile_begin);
           const bool last = (t == sg.tile_end - 1);
@@ -606,8 +644,18 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           if (warp == 6 && lane == 0) MLRA_TRACE_POINT(1, 320 + min((int)it, 31));
           tc_fence_after();
           float s[HW];
-          tmem_load_row<HW>(tbase + lane_base + Sh::S_COL0 + (it % Sh::SBUF) * NP + hcol, s);
-          tmem_ld_wait();
+          const uint32_t s_addr = tbase + lane_base + Sh::S_COL0 + (it % Sh::SBUF) * Sh::MN + hcol;
+          tmem_load_row<HW>(s_addr, s);
+          if constexpr (Sh::FP8) {
+            // score = factor * (S from the hi terms + S from the lo terms)
+            float s_lo[HW];
+            tmem_load_row<HW>(s_addr + NP, s_lo);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < HW; ++x) s[x] = (s[x] + s_lo[x]) * qf[x];
+          } else {
+            tmem_ld_wait();
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sfree_bar[it % Sh::SBUF]);
@@ -647,7 +695,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
           for (int x = 0; x < HW; ++x) pr[x] = fast_exp2(xs[x]);
 
-          const bool need = named_bar_or(bar_or, 128, !okl || first || dmax > kRescaleSlack);
+          const bool need = named_bar_or(bar_or, 128, !okl || first || dmax > Sh::SLACK);
           if (warp == 2 && lane == 0) MLRA_TRACE_POINT(1, 256 + min((int)it, 31));
           if (need) {
             if (named_bar_or(bar_or, 128, !okl || *abort_flag)) { ok = false; break; }
@@ -687,13 +735,16 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
               tc_fence_after();
 #pragma unroll
               for (int mt = 0; mt < Sh::NMT; ++mt) {
-                float o[HW];
-                const uint32_t oa = tbase + lane_base + Sh::O_COL + mt * NP + hcol;
-                tmem_load_row<HW>(oa, o);
-                tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < HW; ++x) o[x] *= alpha[x];
-                tmem_store_row<HW>(oa, o);
+                for (int qt = 0; qt < Sh::NQ; ++qt) {  // every term's columns
+                  float o[HW];
+                  const uint32_t oa = tbase + lane_base + Sh::O_COL + mt * Sh::MN + qt * NP + hcol;
+                  tmem_load_row<HW>(oa, o);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int x = 0; x < HW; ++x) o[x] *= alpha[x];
+                  tmem_store_row<HW>(oa, o);
+                }
               }
               tmem_st_wait();
             }
@@ -704,14 +755,39 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             add_f32x2(l_part[x], l_part[x + 1], l_part[x], l_part[x + 1], pr[x], pr[x + 1]);
           uint8_t* pbuf = Sh::P_IN_STAGE ? stages + (it % STAGES) * Sh::STAGE_BYTES + Sh::NC * Sh::C_REG
                                          : pbufs + (it % max(Sh::PBUF, 1)) * Sh::P_BYTES;
+          if constexpr (Sh::FP8) {
+            // P row = [hi terms of the NP heads | lo terms], E4M3, of p * P_SCALE
+            static_assert(HW % 16 == 0, "16-byte P stores");
 #pragma unroll
-          for (int c = 0; c < HW / 8; ++c) {
-            uint4 w;
-            w.x = pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]);
-            w.y = pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]);
-            w.z = pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]);
-            w.w = pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]);
-            *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + hcol * 2 + c * 16, Sh::P_ROWB)) = w;
+            for (int c = 0; c < HW / 16; ++c) {
+              uint32_t hw[8], lw[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                uint16_t h2, l2;
+                e4m3x2_split(pr[16 * c + 2 * e] * Sh::P_SCALE, pr[16 * c + 2 * e + 1] * Sh::P_SCALE, h2, l2);
+                if (e % 2 == 0) {
+                  hw[e / 2] = h2;
+                  lw[e / 2] = l2;
+                } else {
+                  hw[e / 2] |= static_cast<uint32_t>(h2) << 16;
+                  lw[e / 2] |= static_cast<uint32_t>(l2) << 16;
+                }
+              }
+              *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + hcol + c * 16, Sh::P_ROWB)) =
+                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + NP + hcol + c * 16, Sh::P_ROWB)) =
+                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < HW / 8; ++c) {
+              uint4 w;
+              w.x = pack_bf16x2(pr[8 * c + 0], pr[8 * c + 1]);
+              w.y = pack_bf16x2(pr[8 * c + 2], pr[8 * c + 3]);
+              w.z = pack_bf16x2(pr[8 * c + 4], pr[8 * c + 5]);
+              w.w = pack_bf16x2(pr[8 * c + 6], pr[8 * c + 7]);
+              *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + hcol * 2 + c * 16, Sh::P_ROWB)) = w;
+            }
           }
           if (g == 0 && last && !valid) {
             // rows past the sequence end: zero them so stale or NaN slots cannot reach O
@@ -745,15 +821,23 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
             for (int x = 0; x < HW; ++x) {
               const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
-              inv[x] = 1.f / l;
+              inv[x] = (Sh::FP8 ? p.o_scale : 1.f) / l;
               if (sw == 0 && x % 32 == lane && hcol + x < nheads)
                 p.lse_part[(size_t)slot * p.h + head0 + hcol + x] = m(x) + __log2f(l);
             }
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
               float o[HW];
-              tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * NP + hcol, o);
-              tmem_ld_wait();
+              tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + hcol, o);
+              if constexpr (Sh::FP8) {
+                float o_lo[HW];
+                tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + NP + hcol, o_lo);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < HW; ++x) o[x] += o_lo[x];
+              } else {
+                tmem_ld_wait();
+              }
               const int f = mt * 128 + row;
               if (f < Sh::DB) {
                 float* dst = p.o_part + ((size_t)slot * p.h + head0 + hcol) * Sh::DB + f;

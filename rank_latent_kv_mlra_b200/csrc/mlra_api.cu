@@ -29,7 +29,7 @@ namespace {
 // Compiled kernel set. A variant fixes (d_b, d_rope, heads per CTA, d_h) and the decode
 // kernel's shared-memory pipeline.
 // ---------------------------------------------------------------------------------------
-enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kMlra4Sum = 4, kMlra2Sum = 5, kNumVariants };
+enum Variant { kTiny = 0, kMlra4 = 1, kMlra2 = 2, kMla = 3, kMlra4Sum = 4, kMlra2Sum = 5, kMlra4F8 = 6, kNumVariants };
 
 using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 // P is written over each stage's RoPE columns, which leaves room for two query buffers (the
@@ -44,6 +44,9 @@ using DecMla = DecodeShape<512, 64, 64, 1, 1, 0>;
 // MMA of N = 64 costs the same issue time as N = 32); P lives in each stage's RoPE region so
 // that four 48 KB stages fit next to the 24 KB query
 using DecMlra4Sum = DecodeShape<128, 64, 64, 4, 1, 0>;
+// MLRA-4 over an E4M3 cache: a 128-token stage is 24 KB (128-byte block rows, 64-byte RoPE
+// rows), so six fit beside two 12 KB query buffers (hi and lo terms of 32 heads)
+using DecMlra4F8 = DecodeShape<128, 64, 32, 6, 2, 0, 2, true>;
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 
@@ -52,7 +55,7 @@ struct VariantDims {
 };
 constexpr VariantDims kDims[kNumVariants] = {
     {32, 16, 16, 32}, {128, 64, 32, 128}, {256, 64, 64, 128}, {512, 64, 64, 128}, {128, 64, 64, 128},
-    {256, 64, 64, 128}};
+    {256, 64, 64, 128}, {128, 64, 32, 128}};
 
 // Largest batch tile of the projection kernels: at d_b = 512 a 128-row tile of the merged
 // latent plus W^UV^T would need 256 KB of shared memory.
@@ -84,18 +87,20 @@ CUtensorMapSwizzle swizzle_for(int row_bytes) {
                           : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
 }
 
-// 2-D bf16 tensor [rows][cols] (row stride in bytes), box [box_rows][box_cols].
+// 2-D tensor [rows][cols] of bf16 (esize 2) or bytes (esize 1), row stride in bytes, box
+// [box_rows][box_cols], swizzled by the box's row width.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride,
-              uint32_t box_rows, uint32_t box_cols) {
+              uint32_t box_rows, uint32_t box_cols, int esize = 2) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {row_stride};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_cols * 2),
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_for(box_cols * esize), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -140,6 +145,8 @@ struct mlra_ctx {
   int vh;         // heads of the packed query and partials: h, or k*h when the blocks are summed
   bool summed;    // every head attends to every block; outputs summed
   float alpha;    // alpha_attn (summed blocks)
+  bool fp8;       // E4M3 cache
+  float latent_scale, rope_scale;
   float scale;
   CUtensorMap map_wuk;
   CUtensorMap map_wuv;
@@ -173,6 +180,8 @@ template <int DB, int DH, int NT>
 cudaError_t prep_proj() {
   using S = ProjShape<DB, DH, NT>;
   cudaError_t e = prep_kernel(mlra_absorb_kernel<S>, S::SMEM1);
+  if constexpr (DB == 128 && DH == 128)
+    if (e == cudaSuccess) e = prep_kernel(mlra_absorb_kernel<S, true>, S::SMEM1F8);
   if (e != cudaSuccess) return e;
   e = prep_kernel(mlra_uproj_kernel<S, false>, S::SMEM4);
   if (e != cudaSuccess) return e;
@@ -226,7 +235,7 @@ cudaLaunchConfig_t launch_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s
   return c;
 }
 
-template <int DB, int DH, int NT>
+template <int DB, int DH, int NT, bool F8 = false>
 cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   using S = ProjShape<DB, DH, NT>;
   // a bf16 query is read by TMA: its q^C columns in swizzle-width boxes, its q^R columns in one
@@ -241,9 +250,9 @@ cudaError_t launch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cu
       return cudaErrorInvalidValue;
   }
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t c = launch_cfg(dim3(h->vh, (batch + NT - 1) / NT), dim3(kProjThreads), S::SMEM1, s, true,
-                                    &attr);
-  return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S>, h->map_wuk, mqc, mqr, pp);
+  cudaLaunchConfig_t c = launch_cfg(dim3(h->vh, (batch + NT - 1) / NT), dim3(kProjThreads),
+                                    F8 ? S::SMEM1F8 : S::SMEM1, s, true, &attr);
+  return cudaLaunchKernelEx(&c, mlra_absorb_kernel<S, F8>, h->map_wuk, mqc, mqr, pp);
 }
 template <int DB, int DH, int NT, bool LATENT, int SUMK = 1>
 cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
@@ -255,14 +264,14 @@ cudaError_t launch_uproj(const mlra_ctx* h, const ProjParams& pp, int batch, cud
                                     &attr);
   return cudaLaunchKernelEx(&c, mlra_uproj_kernel<S, LATENT, SUMK>, h->map_wuv, pp);
 }
-template <int DB, int DH>
+template <int DB, int DH, bool F8 = false>
 cudaError_t dispatch_absorb(const mlra_ctx* h, const ProjParams& pp, int batch, cudaStream_t s) {
   switch (nt_for(batch, max_nt<DB>())) {
-    case 16: return launch_absorb<DB, DH, 16>(h, pp, batch, s);
-    case 32: return launch_absorb<DB, DH, 32>(h, pp, batch, s);
-    case 64: return launch_absorb<DB, DH, 64>(h, pp, batch, s);
+    case 16: return launch_absorb<DB, DH, 16, F8>(h, pp, batch, s);
+    case 32: return launch_absorb<DB, DH, 32, F8>(h, pp, batch, s);
+    case 64: return launch_absorb<DB, DH, 64, F8>(h, pp, batch, s);
     default:
-      if constexpr (max_nt<DB>() >= 128) return launch_absorb<DB, DH, 128>(h, pp, batch, s);
+      if constexpr (max_nt<DB>() >= 128) return launch_absorb<DB, DH, 128, F8>(h, pp, batch, s);
       return cudaErrorInvalidValue;
   }
 }
@@ -290,6 +299,7 @@ cudaError_t launch_decode(const mlra_ctx* h, const CUtensorMap& mc, const CUtens
 struct Workspace {
   int* status;
   __nv_bfloat16* q_pack;
+  float* qfac;  // E4M3 cache only
   float* o_part;
   float* lse_part;
   size_t bytes;
@@ -304,7 +314,13 @@ Workspace carve(const mlra_ctx* h, int batch, void* base) {
   w.status = reinterpret_cast<int*>(p + off);
   off += 256;
   w.q_pack = reinterpret_cast<__nv_bfloat16*>(p + off);
+  // bf16 rows, or two E4M3 rows (the hi and lo terms) per head: the same bytes
   off += align256((size_t)batch * h->nsub * h->np * (h->d_b + h->d_r) * 2);
+  w.qfac = nullptr;
+  if (h->fp8) {
+    w.qfac = reinterpret_cast<float*>(p + off);
+    off += align256((size_t)batch * h->nsub * h->np * 4);
+  }
   const size_t slots = (size_t)batch + h->groups;
   w.o_part = reinterpret_cast<float*>(p + off);
   off += align256(slots * h->vh * h->d_b * 4);
@@ -336,16 +352,20 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = h->cfg.d_c + h->d_r;
 
-  // tensor maps over this call's pool and packed-query buffers
-  const int cw = h->d_b < 64 ? h->d_b : 64, rw = h->d_r < 64 ? h->d_r : 64;
+  // tensor maps over this call's pool and packed-query buffers; a box row is at most 128 bytes
+  const int es = h->fp8 ? 1 : 2;  // bytes per cached / packed-query element
+  const int cw = h->d_b * es < 128 ? h->d_b : 128 / es, rw = h->d_r * es < 128 ? h->d_r : 128 / es;
+  const int nq = h->fp8 ? 2 : 1;  // query rows per head (E4M3: hi and lo terms)
   CUtensorMap mc, mr, mqc, mqr;
-  const uint64_t qrows = (uint64_t)batch * h->nsub * h->np;
-  // a head chunk narrower than the MMA's N loads only its real rows
+  const uint64_t qrows = (uint64_t)batch * h->nsub * h->np * nq;
+  // a head chunk narrower than the MMA's N loads only its real rows (bf16 shapes only: the
+  // E4M3 shape's hi and lo rows come as one box, so its chunks are always full)
   const uint32_t q_rows = h->heads_block < h->np ? h->heads_block : h->np;
-  if (!make_map(&mc, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, cw) ||
-      !make_map(&mr, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * 2, kPage, rw) ||
-      !make_map(&mqc, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, q_rows, cw) ||
-      !make_map(&mqr, w.q_pack, qrows, h->d_b + h->d_r, (uint64_t)(h->d_b + h->d_r) * 2, q_rows, rw))
+  const uint64_t qw = h->d_b + h->d_r;
+  if (!make_map(&mc, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * es, kPage, cw, es) ||
+      !make_map(&mr, pool, (uint64_t)num_pages * kPage, D, (uint64_t)D * es, kPage, rw, es) ||
+      !make_map(&mqc, w.q_pack, qrows, qw, qw * es, q_rows * nq, cw, es) ||
+      !make_map(&mqr, w.q_pack, qrows, qw, qw * es, q_rows * nq, rw, es))
     return MLRA_ERR_CUDA;
 
   ProjParams pp = {};
@@ -372,6 +392,10 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   pp.q_heads = h->cfg.h;
   pp.out_heads = h->cfg.h;
   pp.out_scale = h->summed ? h->alpha : 1.f;
+  pp.latent_scale = h->latent_scale;
+  pp.rope_scale = h->rope_scale;
+  pp.qfac = w.qfac;
+  pp.q_rows_per_sub = h->np * nq;
   // the status word's first 4 bytes; the next two words take early errors by call tag
   const EarlyTags tags = {reinterpret_cast<unsigned*>(w.status) + 1, next_call_tag()};
   pp.status = w.status;
@@ -392,6 +416,8 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
   dp.h = h->vh;
   dp.d_c = h->cfg.d_c;
   dp.q_rows = (int)q_rows;
+  dp.qfac = w.qfac;
+  dp.o_scale = h->fp8 ? h->latent_scale / DecMlra4F8::P_SCALE : 1.f;
   dp.o_part = w.o_part;
   dp.lse_part = w.lse_part;
   dp.status = w.status;
@@ -458,6 +484,15 @@ int run_decode(mlra_handle h, const void* q, mlra_dtype q_dtype, const void* poo
       if (e == cudaSuccess)
         e = latent ? dispatch_uproj<256, 128, true>(h, pp, batch, s)
                    : dispatch_uproj<512, 128, false, 2>(h, pp, batch, s);
+      break;
+    case kMlra4F8:
+      e = dispatch_absorb<128, 128, true>(h, pp, batch, s);
+      rec(1);
+      if (e == cudaSuccess) e = launch_decode<DecMlra4F8>(h, mc, mr, mqc, mqr, dp, s);
+      rec(2);
+      if (e == cudaSuccess)
+        e = latent ? dispatch_uproj<128, 128, true>(h, pp, batch, s)
+                   : dispatch_uproj<128, 128, false>(h, pp, batch, s);
       break;
     case kMla:
       e = dispatch_absorb<512, 128>(h, pp, batch, s);
@@ -561,6 +596,15 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
     return MLRA_ERR_UNSUPPORTED;
   if (summed && var == kMlra4) var = kMlra4Sum;
   if (summed && var == kMlra2) var = kMlra2Sum;
+  // E4M3 cache: compiled for the MLRA-4 block shape (d_b 128, d_rope 64, d_h 128), partitioned
+  // heads, whole 32-head chunks
+  if (c.cache_fp8 != 0 && c.cache_fp8 != 1) return MLRA_ERR_INVALID_ARG;
+  const bool fp8 = c.cache_fp8 == 1;
+  if (fp8 && (summed || var != kMlra4 || hb % 32 != 0)) return MLRA_ERR_UNSUPPORTED;
+  if (fp8 && (!(c.latent_scale >= 0.f) || !(c.rope_scale >= 0.f) || !std::isfinite(c.latent_scale) ||
+              !std::isfinite(c.rope_scale)))
+    return MLRA_ERR_INVALID_ARG;
+  if (fp8) var = kMlra4F8;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLRA_ERR_CUDA;
@@ -582,6 +626,9 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
   h->summed = summed;
   h->vh = summed ? c.k * c.h : c.h;
   h->alpha = c.attn_scale > 0.f ? c.attn_scale : 1.0f / sqrtf((float)c.k);
+  h->fp8 = fp8;
+  h->latent_scale = fp8 && c.latent_scale > 0.f ? c.latent_scale : 1.f;
+  h->rope_scale = fp8 && c.rope_scale > 0.f ? c.rope_scale : 1.f;
   h->chunks = (hb + h->np - 1) / h->np;
   h->nsub = c.k * h->chunks;
   h->groups = h->num_sms / h->nsub;
@@ -616,6 +663,11 @@ int mlra_create(const mlra_config* cfg, const void* w_uk, const void* w_uv, mlra
       e = prep_decode<DecMla>();
       if (e == cudaSuccess) e = prep_proj_all<512, 128>();
       h->stages = DecMla::STAGES;
+      break;
+    case kMlra4F8:
+      e = prep_decode<DecMlra4F8>();
+      if (e == cudaSuccess) e = prep_proj_all<128, 128>();
+      h->stages = DecMlra4F8::STAGES;
       break;
     case kMlra2Sum:
       e = prep_decode<DecMlra2>();
@@ -696,9 +748,14 @@ int mlra_append_cache(mlra_handle h, void* pool, int num_pages, const int32_t* p
   if (in_dtype != MLRA_F32 && in_dtype != MLRA_BF16) return MLRA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLRA_OK;
   const int warps = 8;
-  mlra_append_kernel<<<(n_tokens + warps - 1) / warps, warps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<__nv_bfloat16*>(pool), num_pages, page_table, pt_stride, batch, seq_ids, positions, c_new,
-      kr_new, in_dtype == MLRA_F32, n_tokens, h->cfg.d_c, h->d_r, status);
+  if (h->fp8)
+    mlra_append_e4m3_kernel<<<(n_tokens + warps - 1) / warps, warps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint8_t*>(pool), num_pages, page_table, pt_stride, batch, seq_ids, positions, c_new, kr_new,
+        in_dtype == MLRA_F32, n_tokens, h->cfg.d_c, h->d_r, h->latent_scale, h->rope_scale, status);
+  else
+    mlra_append_kernel<<<(n_tokens + warps - 1) / warps, warps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<__nv_bfloat16*>(pool), num_pages, page_table, pt_stride, batch, seq_ids, positions, c_new,
+        kr_new, in_dtype == MLRA_F32, n_tokens, h->cfg.d_c, h->d_r, status);
   return cudaGetLastError() == cudaSuccess ? MLRA_OK : MLRA_ERR_CUDA;
 }
 
@@ -744,7 +801,7 @@ int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w
   }
   if (e != cudaSuccess) return MLRA_ERR_CUDA;
   AppendRowParams ap = {part, kslices, batch, h->cfg.d_c, h->d_r, d_out, positions, page_table, pt_stride,
-                        num_pages, static_cast<__nv_bfloat16*>(pool),
+                        num_pages, pool, h->fp8 ? 1 : 0, h->latent_scale, h->rope_scale,
                         std::log2((double)(rope_base > 1.f ? rope_base : 10000.f)), status, tags};
   const int total = batch * (d_out / 2);
   cudaLaunchAttribute attr;

@@ -7,7 +7,8 @@
 //   k^R = RoPE_pos(x W^KR)     its decoupled positional key, shared by every head (lesty.tech
 //                              section 4), rotated as in RoFormer: pair (2i, 2i+1) by the angle
 //                              pos * base^(-2i / d_r)
-//   row [c | k^R] -> bf16, slot pos % 64 of page page_table[b][pos / 64]
+//   row [c | k^R] -> bf16 (or E4M3 bytes of v / scale for an E4M3 cache), slot pos % 64 of
+//   page page_table[b][pos / 64]
 //
 // Both weight matrices are one bf16 matrix w_down [d_c + d_r][d_model], one row per output
 // feature. Two kernels:
@@ -163,7 +164,9 @@ struct AppendRowParams {
   const int* page_table;  // [batch][pt_stride]
   int pt_stride;
   int num_pages;
-  __nv_bfloat16* pool;    // [num_pages][64][d_out]
+  void* pool;             // [num_pages][64][d_out] bf16, or E4M3 bytes when fp8
+  int fp8;                // E4M3 cache: store e4m3(v / scale)
+  float latent_scale, rope_scale;
   double log2_base;       // log2 of the RoPE base
   int* status;
   EarlyTags tags;         // the down-projection kernel's errors, folded in by block 0
@@ -248,7 +251,13 @@ __global__ void __launch_bounds__(kAppendPairs * kAppendGroups) mlra_rope_append
     v0 = r0;
     v1 = r1;
   }
-  *reinterpret_cast<uint32_t*>(p.pool + ((size_t)page * kPage + pos % kPage) * p.d_out + f0) = pack_bf16x2(v0, v1);
+  const size_t at = ((size_t)page * kPage + pos % kPage) * p.d_out + f0;
+  if (p.fp8) {
+    const float sc = f0 < p.d_c ? p.latent_scale : p.rope_scale;
+    *reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(p.pool) + at) = e4m3x2_from_f32(__fdiv_rn(v0, sc), __fdiv_rn(v1, sc));
+  } else {
+    *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.pool) + at) = pack_bf16x2(v0, v1);
+  }
 }
 
 }  // namespace mlra

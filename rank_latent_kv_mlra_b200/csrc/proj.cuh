@@ -55,6 +55,11 @@ struct ProjParams {
   int q_heads;        // heads of the query rows (head v reads query row v % q_heads)
   int out_heads;      // heads of the output rows
   float out_scale;    // alpha_attn when the blocks are summed, else 1
+  // E4M3 cache (absorb writes each head's query as two E4M3 terms with a power-of-two factor)
+  float latent_scale;  // value of a latent byte = latent_scale * e4m3(byte)
+  float rope_scale;    // value of a RoPE byte = rope_scale * e4m3(byte)
+  float* qfac;         // [B][nsub][np] factor of each head's query terms
+  int q_rows_per_sub;  // query rows per (sequence, decode CTA): np, or 2 * np for two terms
   int* status;        // cleared by absorb CTA (0, 0); written by the combine kernel
   EarlyTags tags;     // absorb errors (the decode kernel folds them into status)
   unsigned long long wait_limit_ns;
@@ -80,6 +85,10 @@ struct ProjShape {
   // operand tiles, reused afterwards to stage the output rows
   static constexpr int STG1 = round_up(OFF_QRS + QRS_BYTES > NT * DB * 2 ? OFF_QRS + QRS_BYTES : NT * DB * 2, 1024);
   static constexpr int SMEM1 = STG1 + 1024 + 256;
+  // E4M3 output: the fp32 query rows [NT][DB + up to 64 RoPE columns] are staged after the
+  // barriers, then each is split into two E4M3 terms
+  static constexpr int OFF_STF = STG1 + 256;
+  static constexpr int SMEM1F8 = OFF_STF + NT * (DB + 64) * 4 + 1024;
   static constexpr int TMEM1 = NMT * NT <= 32 ? 32 : NMT * NT <= 64 ? 64 : NMT * NT <= 128 ? 128 :
                                NMT * NT <= 256 ? 256 : 512;
   // uproj: A = (W^UV_h)^T, MN-major: atoms of AW output columns, each DB rows (K) deep
@@ -103,7 +112,11 @@ struct ProjShape {
 // ---------------------------------------------------------------------------------------
 // absorb
 // ---------------------------------------------------------------------------------------
-template <class Sh>
+// F8: the packed query is written for an E4M3 cache: row [q~ * latent_scale | q^R * rope_scale]
+// (times scale * log2 e) of each (sequence, head) is multiplied by a power of two 2^E that puts
+// its largest magnitude in [128, 256), and stored as two E4M3 terms (hi: the nearest E4M3
+// value, lo: the nearest to the remainder) in rows prow and np + prow; qfac receives 2^-E.
+template <class Sh, bool F8 = false>
 __global__ void __launch_bounds__(kProjThreads, 1)
     mlra_absorb_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_qc,
                        const __grid_constant__ CUtensorMap map_qr, const ProjParams p) {
@@ -117,6 +130,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sh::STG1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  float* stf = reinterpret_cast<float*>(smem + Sh::OFF_STF);  // F8 only: [NT][DB + d_r] fp32
 
   const int head = blockIdx.x;
   const int n0 = blockIdx.y * NT;
@@ -222,6 +237,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           w.w = pack_bf16x2(v[i][6], v[i][7]);
           *reinterpret_cast<uint4*>(Bq + (d8 / Sh::AW) * Sh::B1_REG +
                                     swizzle(bl * Sh::AROWB + (d8 % Sh::AW) * 2, Sh::AROWB)) = w;
+        } else if (F8) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) stf[bl * qw + DB + (d8 - DH) + e] = v[i][e] * p.qscale * p.rope_scale;
         } else if (n0 + bl < p.batch) {
           uint4 w;
           w.x = pack_bf16x2(v[i][0] * p.qscale, v[i][1] * p.qscale);
@@ -287,6 +305,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           f[2 * e] = v.x * p.qscale;
           f[2 * e + 1] = v.y * p.qscale;
         }
+        if constexpr (F8) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) stf[bl * qw + DB + c8 + e] = f[e] * p.rope_scale;
+          continue;
+        }
         uint4 w;
         w.x = pack_bf16x2(f[0], f[1]);
         w.y = pack_bf16x2(f[2], f[3]);
@@ -315,22 +338,68 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         tmem_load_row<COLS>(tbase + lane_base + mt * NT + cg * COLS, v);
         tmem_ld_wait();
         if (c < DB) {
+          if constexpr (F8) {
 #pragma unroll
-          for (int n = 0; n < COLS; ++n)
-            stage_out[(cg * COLS + n) * DB + c] = __float2bfloat16_rn(v[n] * p.qscale);
+            for (int n = 0; n < COLS; ++n) stf[(cg * COLS + n) * qw + c] = v[n] * p.qscale * p.latent_scale;
+          } else {
+#pragma unroll
+            for (int n = 0; n < COLS; ++n)
+              stage_out[(cg * COLS + n) * DB + c] = __float2bfloat16_rn(v[n] * p.qscale);
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (ok) {
+  if (ok && !F8) {
     for (int idx = threadIdx.x; idx < NT * (DB / 8); idx += kProjThreads) {
       const int n = idx / (DB / 8), c8 = (idx % (DB / 8)) * 8;
       const int b = n0 + n;
       if (b < p.batch)
         *reinterpret_cast<uint4*>(p.q_pack + (((size_t)b * p.nsub + sub) * p.np + prow) * qw + c8) =
             *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(A) + n * DB + c8);
+    }
+  }
+  if (ok && F8) {
+    // one warp per batch row: the row's largest magnitude fixes its power of two, then each
+    // lane splits 8 consecutive elements into the two E4M3 terms
+    uint8_t* qp8 = reinterpret_cast<uint8_t*>(p.q_pack);
+    for (int n = warp; n < NT; n += kProjThreads / 32) {
+      const int b = n0 + n;
+      if (b >= p.batch) continue;
+      const float* row = stf + n * qw;
+      float amax = 0.f;
+      for (int i = lane; i < qw; i += 32) amax = fmaxf(amax, fabsf(row[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      int ex = 0;
+      if (amax > 0.f) frexpf(amax, &ex);          // amax in [2^(ex-1), 2^ex)
+      const int e = amax > 0.f ? min(max(8 - ex, -120), 120) : 0;
+      const float up = ldexpf(1.f, e);           // amax * up in [128, 256)
+      const size_t hi_row = ((size_t)b * p.nsub + sub) * p.q_rows_per_sub + prow;
+      const size_t lo_row = hi_row + p.np;
+      for (int c8 = lane * 8; c8 < qw; c8 += 32 * 8) {
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float x0 = row[c8 + 2 * e2] * up, x1 = row[c8 + 2 * e2 + 1] * up;
+          const uint16_t h2 = e4m3x2_from_f32(x0, x1);
+          const uint32_t hf = f16x2_from_e4m3x2(h2);
+          const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hf));
+          const uint16_t l2 = e4m3x2_from_f32(x0 - hv.x, x1 - hv.y);
+          if (e2 % 2 == 0) {
+            hw[e2 / 2] = h2;
+            lw[e2 / 2] = l2;
+          } else {
+            hw[e2 / 2] |= static_cast<uint32_t>(h2) << 16;
+            lw[e2 / 2] |= static_cast<uint32_t>(l2) << 16;
+          }
+        }
+        *reinterpret_cast<uint2*>(qp8 + hi_row * qw + c8) = make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2*>(qp8 + lo_row * qw + c8) = make_uint2(lw[0], lw[1]);
+      }
+      if (lane == 0) p.qfac[((size_t)b * p.nsub + sub) * p.np + prow] = ldexpf(1.f, -e);
     }
   }
   // drain before releasing TMEM and shared memory

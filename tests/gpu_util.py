@@ -19,7 +19,8 @@ TOL_LSE_ABS = 2e-2
 
 
 def make_handle(w: W.Workload, inputs: dict):
-    return M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inputs["w_uk"], inputs["w_uv"])
+    fp8 = dict(cache_fp8=True, latent_scale=W.E4M3_SCALE, rope_scale=W.E4M3_SCALE) if w.cache == "e4m3" else {}
+    return M.mlra_create(w.h, w.d_h, w.d_c, w.d_r, w.k, inputs["w_uk"], inputs["w_uv"], **fp8)
 
 
 def run_decode(handle, inputs: dict, out_dtype=torch.float32, latent=False, workspace=None):
@@ -62,10 +63,15 @@ def workspace_views(handle, ws: torch.Tensor, batch: int):
 
 
 def oracle_full(w: W.Workload, inputs: dict):
-    """Oracle on the exact values the GPU reads (bf16-rounded cache and weights; q as given)."""
-    return O.decode(inputs["q"].double().cpu().numpy(), inputs["w_uk"].double().cpu().numpy(),
-                    inputs["w_uv"].double().cpu().numpy(), inputs["pool"].float().cpu().numpy(),
-                    inputs["page_table"].cpu().numpy(), inputs["seq_lens"].cpu().numpy(), w.k, w.d_r)
+    """Oracle on the exact values the GPU reads (bf16-rounded cache and weights, or the E4M3
+    cache's bytes; q as given)."""
+    args = (inputs["q"].double().cpu().numpy(), inputs["w_uk"].double().cpu().numpy(),
+            inputs["w_uv"].double().cpu().numpy())
+    rest = (inputs["page_table"].cpu().numpy(), inputs["seq_lens"].cpu().numpy(), w.k, w.d_r)
+    if w.cache == "e4m3":
+        from oracle import fp8_cache_oracle as F
+        return F.decode_fp8(*args, inputs["pool"].cpu().numpy(), *rest, W.E4M3_SCALE, W.E4M3_SCALE)
+    return O.decode(*args, inputs["pool"].float().cpu().numpy(), *rest)
 
 
 def errors(got: np.ndarray, ref: np.ndarray) -> dict:

@@ -21,14 +21,19 @@ def _bf16_bits_to_f64(u16: np.ndarray) -> np.ndarray:
     return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def _init(q, w_uk, w_uv, k, d_r, summed):
-    _G.update(q=q, w_uk=w_uk, w_uv=w_uv, k=k, d_r=d_r, summed=summed)
+def _init(q, w_uk, w_uv, k, d_r, summed, e4m3_scales):
+    _G.update(q=q, w_uk=w_uk, w_uv=w_uv, k=k, d_r=d_r, summed=summed, e4m3_scales=e4m3_scales)
 
 
 def _task(args):
     from oracle import mlra_oracle as O
-    b, pages_u16, n = args
-    pool = _bf16_bits_to_f64(pages_u16)
+    b, pages, n = args
+    if _G["e4m3_scales"] is not None:  # E4M3 bytes, dequantized by the FP8-cache oracle
+        from oracle import fp8_cache_oracle as F
+        ls, rs = _G["e4m3_scales"]
+        pool = F.dequantize_pool(pages, pages.shape[-1] - _G["d_r"], ls, rs)
+    else:
+        pool = _bf16_bits_to_f64(pages)
     rows = O.gather_rows(pool, np.arange(pool.shape[0])[None, :], 0, n)
     if _G["summed"]:
         out, lse = O.decode_summed_sequence(_G["q"][b], _G["w_uk"], _G["w_uv"], rows, _G["k"], _G["d_r"])
@@ -53,9 +58,10 @@ def _single_threaded_blas():
                 os.environ[key] = v
 
 
-def oracle_workload(w, inputs, workers=None):
+def oracle_workload(w, inputs, workers=None, e4m3_scales=None):
     """Oracle (out [B][h][d_h], lse) for every sequence and head of workload ``w`` (lse is
-    [B][h], or [B][k][h] for the summed reading), on the exact bf16 values the GPU reads."""
+    [B][h], or [B][k][h] for the summed reading), on the exact values the GPU reads (bf16, or
+    E4M3 bytes with the (latent, RoPE) scales ``e4m3_scales``)."""
     import torch  # the parent holds the inputs as torch tensors (possibly on the GPU)
     q = inputs["q"].double().cpu().numpy()
     w_uk = inputs["w_uk"].double().cpu().numpy()
@@ -71,7 +77,10 @@ def oracle_workload(w, inputs, workers=None):
             n = int(lens[b])
             npg = (n + 63) // 64
             idx = pt[b, :npg].long()
-            pages = pool[idx].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+            if pool.dtype == torch.uint8:
+                pages = pool[idx].contiguous().cpu().numpy()
+            else:
+                pages = pool[idx].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
             yield b, pages, n
 
     out = np.zeros((B, h, d_h))
@@ -79,7 +88,8 @@ def oracle_workload(w, inputs, workers=None):
     workers = workers or max(1, min(16, os.cpu_count() or 1))
     ctx = mp.get_context("spawn")
     with _single_threaded_blas():
-        pool_proc = ctx.Pool(workers, initializer=_init, initargs=(q, w_uk, w_uv, w.k, w.d_r, w.summed))
+        pool_proc = ctx.Pool(workers, initializer=_init,
+                             initargs=(q, w_uk, w_uv, w.k, w.d_r, w.summed, e4m3_scales))
     try:
         for b, o, l in pool_proc.imap_unordered(_task, tasks(), chunksize=1):
             out[b] = o

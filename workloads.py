@@ -9,7 +9,8 @@ What a workload holds (all tensors on the requested device):
 * ``seq_lens``   int32 [B]: context length n_b of each sequence.
 * ``page_table`` int32 [B][max_pages]: logical page i of sequence b -> physical page id.
   Entries past a sequence's last page are -1.
-* ``pool``       bf16 [num_pages][64][d_c + d_r]: the paged latent cache. Row layout per
+* ``pool``       bf16 [num_pages][64][d_c + d_r] (uint8 E4M3 bytes for an ``e4m3`` cache,
+  each meaning ``E4M3_SCALE * e4m3(byte)``): the paged latent cache. Row layout per
   token is ``[c_1 | ... | c_k | k^R]`` (k latent blocks of d_c/k, then the decoupled RoPE
   key). Slots past n_b in a sequence's last page hold NaN, so a kernel that lets unused
   slots leak into its result fails loudly.
@@ -50,6 +51,7 @@ class Workload:
     tiny_scaling: bool = False             # activations / sqrt(width)
     q_dtype: str = "bf16"                  # "bf16" | "f32"
     summed: bool = False                   # every head attends to every block; outputs summed
+    cache: str = "bf16"                    # "bf16" | "e4m3" (one byte per cached element)
 
     @property
     def d_b(self) -> int:
@@ -79,6 +81,9 @@ WORKLOADS = {
         # the batch-64, context-4096 shapes
         Workload("mlra2sum_h128_b64_n4096", k=2, h=128, d_h=128, d_c=512, d_r=64, batch=64,
                  seq_len=4096, seed=7, summed=True),
+        # the headline shapes over an E4M3 cache (latent and RoPE columns scaled by 2^-5)
+        Workload("mlra4fp8_h128_b32_n8192", k=4, h=128, d_h=128, d_c=512, d_r=64, batch=32,
+                 seq_len=8192, seed=8, cache="e4m3"),
         # One rank's share under 4-way tensor parallelism of the model above (h = 128,
         # d_c = 512, d_r = 64): an MLRA-4 rank holds one block plus the RoPE key and its 32
         # heads; an MLA rank holds the whole latent and 32 heads. Batch 64 keeps either cache
@@ -91,6 +96,10 @@ WORKLOADS = {
 }
 
 HEADLINE = "mlra4_h128_b32_n8192"
+
+# Scales of the E4M3 workloads' caches: a cached byte e means E4M3_SCALE * e4m3(e). With N(0,1)
+# values the largest magnitude in a 2.5 GB cache stays far below 448 * 2^-5 = 14.
+E4M3_SCALE = 2.0 ** -5
 
 
 def scaled(w: Workload, **changes) -> Workload:
@@ -186,12 +195,18 @@ def make_workload(w: Workload, device="cpu", seq_lens: Optional[torch.Tensor] = 
     w_uk32 = randn(*wshape) * w_scale
     w_uv32 = randn(*wshape) * w_scale
 
+    if w.cache == "e4m3":
+        # stored bytes: nearest E4M3 value of v / scale (torch's float8_e4m3fn conversion; no
+        # value reaches its range limit at this scale); NaN slots stay NaN (0x7F)
+        pool = (pool32 / E4M3_SCALE).to(torch.float8_e4m3fn).view(torch.uint8)
+    else:
+        pool = pool32.to(torch.bfloat16)
     out = {
         "workload": w,
         "seq_lens": seq_lens,
         "page_table": page_table,
         "num_pages": num_pages,
-        "pool": pool32.to(torch.bfloat16),
+        "pool": pool,
         "q": q32 if w.q_dtype == "f32" else q32.to(torch.bfloat16),
         "w_uk": w_uk32.to(torch.bfloat16),
         "w_uv": w_uv32.to(torch.bfloat16),
