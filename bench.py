@@ -564,6 +564,63 @@ def inp_for_cpu(w, dev):
     return W.make_workload(w, device=dev)
 
 
+def run_tp(args, world, rank, local):
+    """k-way tensor parallelism of the workload's MLRA-k layer across the torchrun ranks
+    (world size = k): rank j decodes latent block j's cache shard for head group j, and the
+    ranks all-gather their heads (NCCL) every step. Timed on the device, max over ranks; value =
+    the whole layer's cache bytes per step / step time."""
+    import rank_latent_kv_mlra_b200 as M
+    from rank_latent_kv_mlra_b200 import tp
+
+    w = W.WORKLOADS[args.workload]
+    if world != w.k or w.summed or w.cache != "bf16":
+        raise SystemExit(f"--tp needs world size = k ({w.k}) and a partitioned bf16 workload")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = W.make_workload(w, device=dev)  # same seed on every rank: the same layer
+    rd = tp.RankDecode(rank, w.k, w.h, w.d_h, w.d_c, w.d_r, inp["w_uk"], inp["w_uv"])
+    pool = tp.shard_pool(inp["pool"], rank, w.k, w.d_c)
+    q = tp.shard_heads(inp["q"], rank, w.k, 1)
+    pt, sl = inp["page_table"], inp["seq_lens"]
+    nbytes = cache_bytes(w, sl.cpu().tolist())
+    del inp
+    torch.cuda.empty_cache()
+    out = torch.empty(w.batch, w.h // w.k, w.d_h, device=dev, dtype=torch.bfloat16)
+    ws = M.alloc_workspace(rd.handle, w.batch, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        rd.decode(q, pool, pt, sl, out, workspace=ws)
+        return tp.gather_heads(out)
+
+    step()
+    torch.cuda.synchronize()
+    if M.mlra_get_status(ws) != 0:
+        raise RuntimeError(f"rank {rank}: decode status {M.mlra_get_status(ws)}")
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": nbytes / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)",
+        "config": dict(config_of(w, world, nbytes), parallelism=f"tp{world}"),
+        "gpu_launches": 3 * args.steps,
+    }), flush=True)
+
+
 def producer_bytes(w, batch, d_model):
     """Algorithmic bytes of the new-row step: bf16 weights [d_c + d_r][d_model] and hidden
     states read once, bf16 rows written, one position and one page-table entry per token."""
@@ -644,6 +701,8 @@ def main():
                     help="skip timing the other configurations (the `workloads` key)")
     ap.add_argument("--producer", action="store_true",
                     help="time the step before decoding (the new cache rows) instead of the decode step")
+    ap.add_argument("--tp", action="store_true",
+                    help="k-way tensor parallelism of the layer across the torchrun ranks (world size = k)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -653,6 +712,8 @@ def main():
             run_reference(args, world, rank)
         elif args.producer:
             run_producer(args, world, rank, local)
+        elif args.tp:
+            run_tp(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

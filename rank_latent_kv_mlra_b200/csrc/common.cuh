@@ -63,17 +63,20 @@ __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 // Timeline trace points. They compile to nothing unless MLRA_TRACE is defined (a profiling
 // build); then point `id` of kernel `k` in this CTA records %globaltimer into g_mlra_trace.
+// A kernel with trace points starts with MLRA_TRACE_INIT, which reads the buffer pointer once.
 #ifdef MLRA_TRACE
 __device__ unsigned long long* g_mlra_trace;
 constexpr int kTracePoints = 512;
-#define MLRA_TRACE_POINT(k, id)                                                              \
-  do {                                                                                       \
-    const unsigned long long ts_ = global_timer_ns();                                        \
-    if (g_mlra_trace != nullptr && (id) < kTracePoints)                                      \
-      g_mlra_trace[((size_t)(k) * 1024 + blockIdx.x + blockIdx.y * gridDim.x) * kTracePoints + \
-                   (id)] = ts_;                                                              \
+#define MLRA_TRACE_INIT unsigned long long* const mlra_trace_buf_ = g_mlra_trace;
+#define MLRA_TRACE_POINT(k, id)                                                                 \
+  do {                                                                                          \
+    const unsigned long long ts_ = global_timer_ns();                                           \
+    if (mlra_trace_buf_ != nullptr && (id) < kTracePoints)                                      \
+      mlra_trace_buf_[((size_t)(k) * 1024 + blockIdx.x + blockIdx.y * gridDim.x) * kTracePoints + \
+                      (id)] = ts_;                                                              \
   } while (0)
 #else
+#define MLRA_TRACE_INIT
 #define MLRA_TRACE_POINT(k, id) \
   do {                          \
   } while (0)
@@ -109,14 +112,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// Suspends the thread until the phase with the given parity has completed or, at most, about
+// kSuspendHintNs has passed (the hint bounds the suspension; completion wakes the thread at
+// once). A long hint keeps waiting warps from spinning through issue slots that the working
+// warps of the SM need.
+constexpr uint32_t kSuspendHintNs = 200000;
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }

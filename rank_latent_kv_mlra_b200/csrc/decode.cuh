@@ -32,11 +32,11 @@
 
 namespace mlra {
 
-constexpr int kPlanBar = 5;  // named barrier of the segment-list hand-off (1..4: softmax groups)
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2, bool FP8_ = false>
+template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2, bool FP8_ = false,
+          int NWG_ = 2>
 struct DecodeShape {
   static constexpr int DB = DB_;      // latent block width d_c / k
   static constexpr int DR = DR_;      // RoPE key width
@@ -53,9 +53,11 @@ struct DecodeShape {
   // p * P_SCALE <= 2^(SLACK + log2 P_SCALE) = 256 stays inside E4M3's range
   static constexpr float SLACK = FP8 ? 3.0f : 8.0f;
   static constexpr float P_SCALE = FP8 ? 32.0f : 1.0f;
-  static constexpr int NWG = 2;       // softmax warpgroups; each owns NP / NWG heads
+  static constexpr int NWG = NWG_;    // softmax warpgroups; each owns NP / NWG heads
   static constexpr int HW = NP / NWG;
   static constexpr int PV_WARP = 2 + 4 * NWG;  // after the softmax warps
+  // named barriers: 1 + 2g and 2 + 2g for softmax warpgroup g, then the segment-list hand-off
+  static constexpr int PLAN_BAR = 2 * NWG + 1;
   static constexpr int THREADS = 32 * (PV_WARP + 1);
   static constexpr int STAGES = STAGES_;
   static constexpr int QBUF = QBUF_;  // query buffers
@@ -120,6 +122,7 @@ struct DecodeShape {
   static constexpr int SMEM_BYTES = OFF_MISC + 64 * 4 + 1024;  // + alignment slack
   static_assert(DB % CW == 0 && DR % RW == 0, "region split");
   static_assert(NP == 16 || NP == 32 || NP == 64, "heads per CTA");
+  static_assert(NWG >= 1 && NWG <= 7 && NP % NWG == 0 && HW % 8 == 0, "softmax warpgroups");
   static_assert(!FP8 || (NMT == 1 && MN <= 128 && R_ROWB == 64), "E4M3 shapes: one PV M tile, 64-byte RoPE rows");
   static_assert(QBUF == 1 || QBUF == 2, "query buffers");
   static_assert(SBUF >= 2 && TMEM_USED <= 512, "S buffers");
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                        const __grid_constant__ CUtensorMap map_qr, const DecodeParams p) {
   constexpr int NP = Sh::NP, STAGES = Sh::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  MLRA_TRACE_INIT
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem + Sh::OFF_STAGES;
@@ -368,9 +372,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
       }
       __threadfence_block();
       __syncwarp();
-      named_bar_arrive(kPlanBar, Sh::THREADS);
+      named_bar_arrive(Sh::PLAN_BAR, Sh::THREADS);
     } else {
-      named_bar_sync(kPlanBar, Sh::THREADS);
+      named_bar_sync(Sh::PLAN_BAR, Sh::THREADS);
       first_total = plan_words[0];
       first_rb = plan_words[1];
       first_rp = plan_words[2];
@@ -756,15 +760,15 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           uint8_t* pbuf = Sh::P_IN_STAGE ? stages + (it % STAGES) * Sh::STAGE_BYTES + Sh::NC * Sh::C_REG
                                          : pbufs + (it % max(Sh::PBUF, 1)) * Sh::P_BYTES;
           if constexpr (Sh::FP8) {
-            // P row = [hi terms of the NP heads | lo terms], E4M3, of p * P_SCALE
-            static_assert(HW % 16 == 0, "16-byte P stores");
+            // P row = [hi terms of the NP heads | lo terms], E4M3, of p * P_SCALE; 8 heads per
+            // 8-byte store (a swizzle moves whole 16-byte chunks, so 8 aligned bytes stay together)
 #pragma unroll
-            for (int c = 0; c < HW / 16; ++c) {
-              uint32_t hw[8], lw[8];
+            for (int c = 0; c < HW / 8; ++c) {
+              uint32_t hw[2], lw[2];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 4; ++e) {
                 uint16_t h2, l2;
-                e4m3x2_split(pr[16 * c + 2 * e] * Sh::P_SCALE, pr[16 * c + 2 * e + 1] * Sh::P_SCALE, h2, l2);
+                e4m3x2_split(pr[8 * c + 2 * e] * Sh::P_SCALE, pr[8 * c + 2 * e + 1] * Sh::P_SCALE, h2, l2);
                 if (e % 2 == 0) {
                   hw[e / 2] = h2;
                   lw[e / 2] = l2;
@@ -773,10 +777,10 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
                   lw[e / 2] |= static_cast<uint32_t>(l2) << 16;
                 }
               }
-              *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + hcol + c * 16, Sh::P_ROWB)) =
-                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
-              *reinterpret_cast<uint4*>(pbuf + swizzle(row * Sh::P_ROWB + NP + hcol + c * 16, Sh::P_ROWB)) =
-                  make_uint4(lw[0], lw[1], lw[2], lw[3]);
+              *reinterpret_cast<uint2*>(pbuf + swizzle(row * Sh::P_ROWB + hcol + c * 8, Sh::P_ROWB)) =
+                  make_uint2(hw[0], hw[1]);
+              *reinterpret_cast<uint2*>(pbuf + swizzle(row * Sh::P_ROWB + NP + hcol + c * 8, Sh::P_ROWB)) =
+                  make_uint2(lw[0], lw[1]);
             }
           } else {
 #pragma unroll

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
   static_assert(NT * DB * 2 <= Sh::OFF_QRS, "output staging must not overlap the q^R staging");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  MLRA_TRACE_INIT
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* A = smem;
@@ -432,6 +433,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     mlra_uproj_kernel(const __grid_constant__ CUtensorMap map_wuv, const ProjParams p) {
   constexpr int DB = Sh::DB, DH = Sh::DH, NT = Sh::NT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  MLRA_TRACE_INIT
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* A = smem;

@@ -63,6 +63,9 @@ def oracle_workload(w, inputs, workers=None, e4m3_scales=None):
     [B][h], or [B][k][h] for the summed reading), on the exact values the GPU reads (bf16, or
     E4M3 bytes with the (latent, RoPE) scales ``e4m3_scales``)."""
     import torch  # the parent holds the inputs as torch tensors (possibly on the GPU)
+    if e4m3_scales is None and getattr(w, "cache", "bf16") == "e4m3":
+        import workloads
+        e4m3_scales = (workloads.E4M3_SCALE, workloads.E4M3_SCALE)
     q = inputs["q"].double().cpu().numpy()
     w_uk = inputs["w_uk"].double().cpu().numpy()
     w_uv = inputs["w_uv"].double().cpu().numpy()

@@ -33,36 +33,25 @@ def _gpu():
     M.load_library()
 
 
-def rank_shard(w, inp, j):
-    """Rank j's inputs: cache columns [c_j | k^R] (a page pool of its own), the head group's
-    query rows and up-projections. Test-side data layout only."""
-    d_b, hb = w.d_c // w.k, w.h // w.k
-    pool = torch.cat([inp["pool"][..., j * d_b:(j + 1) * d_b], inp["pool"][..., w.d_c:]], dim=-1).contiguous()
-    return {
-        "pool": pool,
-        "page_table": inp["page_table"],
-        "seq_lens": inp["seq_lens"],
-        "q": inp["q"][:, j * hb:(j + 1) * hb].contiguous(),
-        "w_uk": inp["w_uk"][j * hb:(j + 1) * hb].contiguous(),
-        "w_uv": inp["w_uv"][j * hb:(j + 1) * hb].contiguous(),
-    }
-
-
 @pytest.mark.parametrize("name", list(CASES))
 def test_rank_shards_concatenate_to_the_layer_output(name):
+    """Each rank's shard is cut by the library's tp helpers and decoded by tp.RankDecode."""
+    from rank_latent_kv_mlra_b200 import tp
     w = CASES[name]
     inp = W.make_workload(w, device="cuda")
-    d_b, hb = w.d_c // w.k, w.h // w.k
     outs, lses = [], []
     for j in range(w.k):
-        sh = rank_shard(w, inp, j)
-        hdl = M.mlra_create(hb, w.d_h, d_b, w.d_r, 1, sh["w_uk"], sh["w_uv"],
-                            softmax_scale=1.0 / (w.d_h + w.d_r) ** 0.5)
-        out, lse, ws = G.run_decode(hdl, sh)
+        rank = tp.RankDecode(j, w.k, w.h, w.d_h, w.d_c, w.d_r, inp["w_uk"], inp["w_uv"])
+        pool_j = tp.shard_pool(inp["pool"], j, w.k, w.d_c)
+        q_j = tp.shard_heads(inp["q"], j, w.k, 1)
+        out = torch.full((w.batch, w.h // w.k, w.d_h), float("nan"), device="cuda")
+        lse = torch.full((w.batch, w.h // w.k), float("nan"), device="cuda")
+        ws = rank.decode(q_j, pool_j, inp["page_table"], inp["seq_lens"], out, lse)
+        torch.cuda.synchronize()
         assert M.mlra_get_status(ws) == 0
         outs.append(out)
         lses.append(lse)
-        del hdl
+        del rank
     out = torch.cat(outs, dim=1).cpu().numpy()
     lse = torch.cat(lses, dim=1).cpu().numpy()
     ref = G.oracle_full(w, inp)
