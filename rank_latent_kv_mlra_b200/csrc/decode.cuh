@@ -36,7 +36,7 @@ namespace mlra {
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int DB_, int DR_, int NP_, int STAGES_, int QBUF_, int PBUF_, int SBUF_ = 2, bool FP8_ = false,
-          int NWG_ = 2>
+          int NWG_ = 2, int TPS_ = 1>
 struct DecodeShape {
   static constexpr int DB = DB_;      // latent block width d_c / k
   static constexpr int DR = DR_;      // RoPE key width
@@ -60,6 +60,12 @@ struct DecodeShape {
   static constexpr int PLAN_BAR = 2 * NWG + 1;
   static constexpr int THREADS = 32 * (PV_WARP + 1);
   static constexpr int STAGES = STAGES_;
+  // Tiles per pipeline stage: a stage is TPS consecutive tile slots loaded and freed through
+  // one barrier phase (a phase per 128-token tile costs more than the copies of a small tile
+  // need). Slot i of the ring holds tile i's pages; the last tile of a launch may leave a
+  // stage part-filled.
+  static constexpr int TPS = TPS_;
+  static constexpr int SLOTS = STAGES * TPS;
   static constexpr int QBUF = QBUF_;  // query buffers
   // probability buffers; 0: P(i) is written over the RoPE columns of tile i's own stage,
   // which QK(i) has finished reading when the softmax sees S(i), and the stage is only
@@ -70,7 +76,7 @@ struct DecodeShape {
   // STAGES) has freed tile i's stage, so with at least STAGES slots no ring slot is armed again
   // before the phase it held has been waited for (no parity aliasing), however far the softmax
   // runs ahead of the PV issuer.
-  static constexpr int PR = STAGES > 2 ? STAGES : 2;
+  static constexpr int PR = SLOTS > 2 ? SLOTS : 2;
   // A cache row is split into swizzle-width regions (at most 128 bytes): block columns and RoPE
   // columns.
   static constexpr int CW = DB * EB < 128 ? DB : 128 / EB;
@@ -105,7 +111,7 @@ struct DecodeShape {
   static constexpr int MAX_SEGS = 64;
   // small shared state after the big buffers
   static constexpr int OFF_STAGES = 0;
-  static constexpr int OFF_Q = OFF_STAGES + STAGES * STAGE_BYTES;
+  static constexpr int OFF_Q = OFF_STAGES + SLOTS * STAGE_BYTES;
   static constexpr int OFF_P = OFF_Q + QBUF * Q_BYTES;
   // The running max per head is the same in every softmax thread. With 32 heads per warpgroup
   // each warp keeps one copy in shared memory (read as broadcasts, written only when raised),
@@ -233,6 +239,21 @@ __device__ __forceinline__ void shape_mma(uint32_t d, uint64_t a, uint64_t b, ui
     umma_bf16(d, a, b, idesc, acc);
 }
 
+// Ring position of tile i: its slot (shared-memory tile), its stage (barriers) and the parity
+// of the stage's phase that carries it.
+template <class Sh>
+__device__ __forceinline__ uint32_t tile_slot(uint32_t i) {
+  return ((i / Sh::TPS) % Sh::STAGES) * Sh::TPS + i % Sh::TPS;
+}
+template <class Sh>
+__device__ __forceinline__ uint32_t tile_stage(uint32_t i) {
+  return (i / Sh::TPS) % Sh::STAGES;
+}
+template <class Sh>
+__device__ __forceinline__ uint32_t tile_phase(uint32_t i) {
+  return ((i / Sh::TPS) / Sh::STAGES) & 1;
+}
+
 template <class Sh>
 __global__ void __launch_bounds__(Sh::THREADS, 1)
     mlra_decode_kernel(const __grid_constant__ CUtensorMap map_c,
@@ -279,7 +300,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES * Sh::NG; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], Sh::TPS);  // one arrival per tile of the stage
       mbar_init(&empty_bar[s], 1);
     }
     for (int s = 0; s < Sh::QBUF; ++s) {
@@ -459,12 +480,13 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           if (lane == 0) {
             if (id0 < 0 || id0 >= p.num_pages) { set_status(p.status, kErrPageOob); id0 = 0; }
             if (npg == 2 && (id1 < 0 || id1 >= p.num_pages)) { set_status(p.status, kErrPageOob); id1 = 0; }
-            const int st = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1;
-            uint8_t* dst = stages + st * Sh::STAGE_BYTES;
+            const int st = tile_stage<Sh>(it);
+            const uint32_t ph = tile_phase<Sh>(it);
+            uint8_t* dst = stages + tile_slot<Sh>(it) * Sh::STAGE_BYTES;
             for (int g = 0; g < Sh::NG && ok; ++g) {
               const int gi = st * Sh::NG + g;
-              ok = mbar_wait(&empty_bar[gi], ph ^ 1, abort_flag, p.wait_limit_ns);
+              // the stage's previous phase must be freed before its first tile is loaded
+              if (it % Sh::TPS == 0) ok = mbar_wait(&empty_bar[gi], ph ^ 1, abort_flag, p.wait_limit_ns);
               if (ok && !(p.inject_stall == 1 && it == 0)) {
                 if (g == 0) MLRA_TRACE_POINT(1, 8 + min((int)it, 31));
                 mbar_arrive_expect_tx(&full_bar[gi], npg * Sh::group_tx(g));
@@ -486,6 +508,13 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }
       }
+      // A launch whose last tile leaves its stage part-filled completes that stage's phase with
+      // count-only arrivals (the QK issuer waits for it; the teardown drains it).
+      if (Sh::TPS > 1 && lane == 0 && it % Sh::TPS != 0 && (!more || *abort_flag)) {
+        const int st = tile_stage<Sh>(it - 1);
+        for (int g = 0; g < Sh::NG; ++g)
+          for (uint32_t x = it % Sh::TPS; x < (uint32_t)Sh::TPS; ++x) mbar_arrive(&full_bar[st * Sh::NG + g]);
+      }
     } else if (warp == 1) {
       // ============================== QK issuer ==============================
       // One thread issues S^T(i) = [c_j | k^R](i) [q~ | q^R]^T once tile i's pages (and, at a
@@ -505,14 +534,14 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             if (ci >= Sh::SBUF)
               ok = mbar_wait(&sfree_bar[ci % Sh::SBUF], ((ci / Sh::SBUF) - 1) & 1, abort_flag, p.wait_limit_ns);
             MLRA_TRACE_POINT(1, 432 + min((int)ci, 31));
-            const uint32_t st_addr = smem_u32(stages + (ci % STAGES) * Sh::STAGE_BYTES);
+            const uint32_t st_addr = smem_u32(stages + tile_slot<Sh>(ci) * Sh::STAGE_BYTES);
             const uint32_t q_addr = smem_u32(qbufs + qb * Sh::Q_BYTES);
             const uint32_t d = tbase + Sh::S_COL0 + (ci % Sh::SBUF) * Sh::MN;
             uint32_t acc = 0;
             // each column group's MMAs go out as soon as that group has landed
 #pragma unroll
             for (int g = 0; g < Sh::NG; ++g) {
-              if (ok) ok = mbar_wait(&full_bar[(ci % STAGES) * Sh::NG + g], (ci / STAGES) & 1, abort_flag, p.wait_limit_ns);
+              if (ok) ok = mbar_wait(&full_bar[tile_stage<Sh>(ci) * Sh::NG + g], tile_phase<Sh>(ci), abort_flag, p.wait_limit_ns);
               if (!ok) break;
               if (g == 0) MLRA_TRACE_POINT(1, 400 + min((int)ci, 31));
               tc_fence_after();
@@ -574,7 +603,9 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             tc_fence_after();
             MLRA_TRACE_POINT(1, 72 + min((int)pi, 31));
             const bool first = t == sg.tile_begin;
-            const uint32_t st_addr = smem_u32(stages + (pi % STAGES) * Sh::STAGE_BYTES);
+            const uint32_t st_addr = smem_u32(stages + tile_slot<Sh>(pi) * Sh::STAGE_BYTES);
+            // the stage is freed after its last tile (or the launch's last tile)
+            const bool frees = pi % Sh::TPS == Sh::TPS - 1 || (!more && si == nseg - 1 && t == sg.tile_end - 1);
             const uint32_t p_addr = Sh::P_IN_STAGE ? st_addr + Sh::NC * Sh::C_REG
                                                    : smem_u32(pbufs + (pi % max(Sh::PBUF, 1)) * Sh::P_BYTES);
 #pragma unroll
@@ -589,7 +620,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
               }
               // this M tile's columns are read: its group may be reloaded (the last group also
               // holds the RoPE columns and P, read by every M tile)
-              umma_commit(&empty_bar[(pi % STAGES) * Sh::NG + mt]);
+              if (frees) umma_commit(&empty_bar[tile_stage<Sh>(pi) * Sh::NG + mt]);
             }
             umma_commit(&pvdone_bar[pi % Sh::PR]);
           }
@@ -757,7 +788,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
 #pragma unroll
           for (int x = 0; x < HW; x += 2)
             add_f32x2(l_part[x], l_part[x + 1], l_part[x], l_part[x + 1], pr[x], pr[x + 1]);
-          uint8_t* pbuf = Sh::P_IN_STAGE ? stages + (it % STAGES) * Sh::STAGE_BYTES + Sh::NC * Sh::C_REG
+          uint8_t* pbuf = Sh::P_IN_STAGE ? stages + tile_slot<Sh>(it) * Sh::STAGE_BYTES + Sh::NC * Sh::C_REG
                                          : pbufs + (it % max(Sh::PBUF, 1)) * Sh::P_BYTES;
           if constexpr (Sh::FP8) {
             // P row = [hi terms of the NP heads | lo terms], E4M3, of p * P_SCALE; 8 heads per
@@ -795,7 +826,7 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
           }
           if (g == 0 && last && !valid) {
             // rows past the sequence end: zero them so stale or NaN slots cannot reach O
-            uint8_t* st = stages + (it % STAGES) * Sh::STAGE_BYTES;
+            uint8_t* st = stages + tile_slot<Sh>(it) * Sh::STAGE_BYTES;
 #pragma unroll
             for (int r = 0; r < Sh::NC; ++r)
 #pragma unroll

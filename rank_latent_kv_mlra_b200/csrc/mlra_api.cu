@@ -44,10 +44,10 @@ using DecMla = DecodeShape<512, 64, 64, 1, 1, 0>;
 // MMA of N = 64 costs the same issue time as N = 32); P lives in each stage's RoPE region so
 // that four 48 KB stages fit next to the 24 KB query
 using DecMlra4Sum = DecodeShape<128, 64, 64, 4, 1, 0>;
-// MLRA-4 over an E4M3 cache: a 128-token stage is 24 KB (128-byte block rows, 64-byte RoPE
-// rows), so eight fit beside two 12 KB query buffers (hi and lo terms of 32 heads); three S
-// buffers
-using DecMlra4F8 = DecodeShape<128, 64, 32, 8, 2, 0, 3, true, 2>;
+// MLRA-4 over an E4M3 cache: a 128-token tile is 24 KB (128-byte block rows, 64-byte RoPE
+// rows), so eight fit beside two 12 KB query buffers (hi and lo terms of 32 heads), loaded and
+// freed two tiles per barrier phase (four stages); three S buffers
+using DecMlra4F8 = DecodeShape<128, 64, 32, 4, 2, 0, 3, true, 2, 2>;
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 
