@@ -125,7 +125,7 @@ int mlra_workspace_size(mlra_handle h, int batch, size_t* bytes);
  *   lse        device fp32 [batch][h] natural-log log-sum-exp of the scaled scores, or NULL.
  *   workspace  device, >= mlra_workspace_size(batch) bytes, 256-byte aligned. Its first
  *              4 bytes become this call's status word (the first kernel clears it once the
- *              kernel before it in the stream has finished); the next 8 bytes take errors
+ *              kernel before it in the stream has finished); the next 16 bytes take errors
  *              found before that clear, which a later kernel of the call folds into it.
  * Launches three kernels on `stream`: query absorption, split-KV latent attention, and
  * log-sum-exp combine fused with the W^UV up-projection. All three use programmatic

@@ -17,6 +17,10 @@ constexpr int kTile = 128;   // tokens per decode tile (two pages, the MMA M ext
 // Device status codes (same values as mlra_status).
 enum : int { kOk = 0, kErrPageOob = -4, kErrTimeout = -5, kErrSeqLen = -7, kErrDrain = -9 };
 
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 // First error wins.
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
@@ -32,25 +36,37 @@ __device__ __forceinline__ void force_status(int* status, int code) {
 // they store the call's tag (a number unique to each host call, never 0) into a tag word of
 // the workspace, one word per error kind, and a later kernel of the same call, which runs
 // after the first has completed, turns a matching tag into the status code. A tag left in
-// the word by an earlier call never matches. tags[0]: pipeline wait timed out; tags[1]:
-// teardown drain failed.
+// the word by an earlier call never matches.
 struct EarlyTags {
-  unsigned* words;  // 2 words in the call's workspace
+  unsigned* words;  // 4 words in the call's workspace (kinds below)
   unsigned tag;     // this call's tag
 };
+enum : int { kTagTimeout = 0, kTagDrain = 1, kTagSeqLen = 2, kTagPageOob = 3 };
 __device__ __forceinline__ void report_early(const EarlyTags& t, int which) {
   if (t.words != nullptr) atomicExch(t.words + which, t.tag);
+}
+// The first kernel's clearing CTA: status word to 0, and every tag word that does not hold
+// this call's tag to 0 (a compare-and-swap, so a tag another CTA has just written survives;
+// afterwards no word holds stale bits that could equal a later call's tag).
+__device__ __forceinline__ void clear_status_and_tags(int* status, const EarlyTags& t) {
+  if (status != nullptr) *status = 0;
+  if (t.words == nullptr) return;
+  for (int k = 0; k < 4; ++k) {
+    const unsigned w = *reinterpret_cast<volatile unsigned*>(t.words + k);
+    if (w != t.tag) atomicCAS(t.words + k, w, 0u);
+  }
 }
 // Called by one thread of a later kernel of the same call, after griddepcontrol.wait.
 __device__ __forceinline__ void fold_early(const EarlyTags& t, int* status) {
   if (t.words == nullptr) return;
-  const unsigned* w = t.words;
-  if (*reinterpret_cast<const volatile unsigned*>(w + 1) == t.tag) force_status(status, kErrDrain);
-  else if (*reinterpret_cast<const volatile unsigned*>(w) == t.tag) set_status(status, kErrTimeout);
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  const volatile unsigned* w = t.words;
+  if (w[kTagDrain] == t.tag) {
+    force_status(status, kErrDrain);
+    return;
+  }
+  if (w[kTagTimeout] == t.tag) set_status(status, kErrTimeout);
+  if (w[kTagSeqLen] == t.tag) set_status(status, kErrSeqLen);
+  if (w[kTagPageOob] == t.tag) set_status(status, kErrPageOob);
 }
 
 __device__ __forceinline__ uint64_t global_timer_ns() {

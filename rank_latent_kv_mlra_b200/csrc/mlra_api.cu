@@ -782,17 +782,17 @@ int mlra_project_append(mlra_handle h, const void* x, int d_model, const void* w
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MLRA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  g_use_pdl = true;
   const int nt = nt_for(batch, 128);
   const int kslices = d_model / kProjSlice;
   CUtensorMap mw, mx;
   if (!make_map(&mw, w_down, (uint64_t)d_out, (uint64_t)d_model, (uint64_t)d_model * 2, 128, 64) ||
       !make_map(&mx, x, (uint64_t)batch, (uint64_t)d_model, (uint64_t)d_model * 2, (uint32_t)nt, 64))
     return MLRA_ERR_CUDA;
-  int* status = static_cast<int*>(workspace);
   float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 256);
   const EarlyTags tags = {reinterpret_cast<unsigned*>(status) + 1, next_call_tag()};
   DownParams dp = {d_out, batch, part, status, tags, kWaitLimitNs};
-  g_use_pdl = true;
   cudaError_t e;
   switch (nt) {
     case 16: e = launch_down_proj<16>(mw, mx, dp, d_out, kslices, batch, s); break;

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(Sh::THREADS)
     for (int r = 0; r < Sh::NKR; ++r)
       tma_load_2d(A + r * Sh::A_REG, &map_w, &bars[0], ks * Sh::KS + r * 64, mt * 128, pol_w);
     grid_dependency_wait();
-    if (mt == 0 && ks == 0 && blockIdx.z == 0 && p.status) *p.status = 0;
+    if (mt == 0 && ks == 0 && blockIdx.z == 0) clear_status_and_tags(p.status, p.tags);
     const uint64_t pol_x = l2_policy_evict_last();  // every 128-feature tile reads the same x
     for (int r = 0; r < Sh::NKR; ++r)
       tma_load_2d(B + r * Sh::B_REG, &map_x, &bars[0], ks * Sh::KS + r * 64, n0, pol_x);
@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(Sh::THREADS)
   tc_fence_before();
   __syncthreads();
   // this kernel may fail before CTA (0, 0, 0) has cleared the status word: report by tag
-  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, 0);
-  if (threadIdx.x == 0 && !drained) report_early(p.tags, 1);
+  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, kTagTimeout);
+  if (threadIdx.x == 0 && !drained) report_early(p.tags, kTagDrain);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM);

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       for (int r0 = 0; r0 < Sh::NMT * 128; r0 += Sh::A1_BOXR)
         tma_load_2d(A + kr * Sh::A1_REG + r0 * Sh::AROWB, &map_wuk, &bars[0], kr * Sh::AW, head * DB + r0, pol);
     grid_dependency_wait();
-    if (blockIdx.x == 0 && blockIdx.y == 0 && p.status) *p.status = 0;
+    if (blockIdx.x == 0 && blockIdx.y == 0) clear_status_and_tags(p.status, p.tags);
     if (tma_q) {
       const int qh = head % p.q_heads;
       for (int kr = 0; kr < Sh::NKR; ++kr)
@@ -413,8 +413,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   tc_fence_before();
   __syncthreads();
   // this kernel may fail before CTA (0, 0) has cleared the status word: report by tag
-  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, 0);
-  if (threadIdx.x == 0 && !drained) report_early(p.tags, 1);
+  if (threadIdx.x == 0 && *abort_flag) report_early(p.tags, kTagTimeout);
+  if (threadIdx.x == 0 && !drained) report_early(p.tags, kTagDrain);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, Sh::TMEM1);

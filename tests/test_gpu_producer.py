@@ -125,3 +125,27 @@ def test_decode_reads_the_appended_row():
     assert M.mlra_get_status(ws) == 0
     ref = G.oracle_full(w, inp)
     G.assert_parity(out.cpu().numpy(), ref["out"], "decode after append")
+
+
+def test_e4m3_cache_rows():
+    """New rows into an E4M3 cache: each stored byte is the E4M3 value nearest to row / scale
+    (the GPU rounds its fp32 sum, the oracle its float64 value, so a value within the fp32
+    accumulation error of a rounding midpoint may take the neighbouring code: one E4M3 step at
+    most); nothing else in the pool changes."""
+    from oracle import fp8_cache_oracle as F
+    w = W.scaled(W.WORKLOADS["mlra4fp8_h128_b32_n8192"], batch=5, seq_len=None, len_range=(1, 700), seed=56)
+    inp = W.make_workload(w, device="cuda")
+    pr = W.make_producer_inputs(w, inp, d_model=384)
+    before = inp["pool"].clone()
+    assert _run(w, inp, pr) == 0
+    rows, pages, slots = _oracle_rows(w, inp, pr)
+    pool = inp["pool"]
+    pi, si = torch.as_tensor(pages, device="cuda").long(), torch.as_tensor(slots, device="cuda").long()
+    got = pool[pi, si].cpu().numpy()
+    deq = F.e4m3_decode_array(got) * W.E4M3_SCALE
+    assert np.all(np.abs(deq - rows) <= np.abs(rows) * 2.0 ** -3 + W.E4M3_SCALE * 2.0 ** -9)
+    exact = F.quantize_rows(rows, w.d_c, W.E4M3_SCALE, W.E4M3_SCALE)
+    assert np.mean(got == exact) > 0.99
+    mask = torch.ones(pool.shape[:2], dtype=torch.bool, device="cuda")
+    mask[pi, si] = False
+    assert torch.equal(pool[mask], before[mask])
