@@ -72,33 +72,48 @@ def decode_flops(w, seq_lens):
     return float(sum(int(n) for n in seq_lens)) * heads * (2 * (d_b + w.d_r) + 2 * d_b)
 
 
-def kernel_source_hash():
-    """Hash of the decode kernel's code (comments and blank lines left out, so a comment edit
-    does not invalidate a recorded ncu capture)."""
+def decode_shape_name(w):
+    """The decode kernel shape (`using Dec...` in mlra_api.cu) a workload runs on."""
+    d_b = w.d_c // w.k
+    if w.cache == "e4m3":
+        return "DecMlra4F8"
+    if d_b == 32:
+        return "DecTiny"
+    if d_b == 128:
+        return "DecMlra4Sum" if w.summed else "DecMlra4"
+    if d_b == 256:
+        return "DecMlra2"
+    return "DecMla"
+
+
+def kernel_source_hash(w):
+    """Hash of the decode kernel code workload `w` runs: common.cuh, decode.cuh and the line of
+    mlra_api.cu that fixes its shape (comments and blank lines left out, so a comment edit or
+    another shape's change does not invalidate a recorded ncu capture)."""
     h = hashlib.sha256()
+    shape = decode_shape_name(w)
     for f in ["common.cuh", "decode.cuh", "mlra_api.cu"]:
         with open(os.path.join(ROOT, "rank_latent_kv_mlra_b200", "csrc", f), encoding="utf-8") as fh:
             for line in fh:
                 code = line.split("//", 1)[0].rstrip()
-                # of the API file only the decode kernel's compiled shapes count
-                if code and (f != "mlra_api.cu" or code.startswith("using Dec")):
+                if code and (f != "mlra_api.cu" or code.startswith(f"using {shape} ")):
                     h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload_name):
-    """DRAM bytes per launch of the decode kernel from a committed ncu summary, if the kernel
-    source has not changed since it was captured."""
+    """DRAM bytes per launch of the decode kernel from a committed ncu summary, if the code of
+    the kernel the workload runs has not changed since it was captured."""
     path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_source_hash") != kernel_source_hash():
-        return None
     ent = rec.get("workloads", {}).get(workload_name)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    if ent is None or ent.get("kernel_source_hash") != kernel_source_hash(W.WORKLOADS[workload_name]):
+        return None
+    return ent.get("dram_bytes_per_launch")
 
 
 class ClockSampler:

@@ -35,7 +35,9 @@ using DecTiny = DecodeShape<32, 16, 16, 4, 2, 2>;
 // P is written over each stage's RoPE columns, which leaves room for two query buffers (the
 // next segment's query loads while the current one is in use)
 using DecMlra4 = DecodeShape<128, 64, 32, 4, 2, 0>;
-using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 1>;
+// MLRA-2 (and summed MLRA-2): two 80 KB stages beside the 40 KB query; P is written over each
+// stage's RoPE columns, so the next tile's softmax does not wait for this tile's P.C
+using DecMlra2 = DecodeShape<256, 64, 64, 2, 1, 0>;
 // MLA (k = 1): a 128-token stage of whole 1152-byte rows is 144 KB, so one stage fits; 64
 // heads per CTA (2 CTAs per group) halve the MMA work per cached byte against 32, and P goes
 // into the stage so the 72 KB query fits beside it
