@@ -852,14 +852,21 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             warp_reduce_scatter<HW, false>(lt, lane);
             store_scattered<HW>(lt, red + q4 * HW, lane);
             named_bar_sync(bar_sync, 128);
+            // This runs while the next segment's tiles wait behind it, so it is kept short: an
+            // approximate reciprocal (l >= 1: the running maximum's own term contributes 1, so
+            // the 2-ulp bound of div.approx holds) and one lse store per warp, lane x holding
+            // head x, instead of one single-lane store per head.
+            static_assert(HW <= 32, "one lse lane per head");
             float inv[HW];
+            float lse_lane = 0.f;
 #pragma unroll
             for (int x = 0; x < HW; ++x) {
               const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
-              inv[x] = (Sh::FP8 ? p.o_scale : 1.f) / l;
-              if (sw == 0 && x % 32 == lane && hcol + x < nheads)
-                p.lse_part[(size_t)slot * p.h + head0 + hcol + x] = m(x) + __log2f(l);
+              inv[x] = __fdividef(Sh::FP8 ? p.o_scale : 1.f, l);
+              if (x == lane) lse_lane = m(x) + __log2f(l);
             }
+            if (sw == 0 && lane < HW && hcol + lane < nheads)
+              p.lse_part[(size_t)slot * p.h + head0 + hcol + lane] = lse_lane;
 #pragma unroll
             for (int mt = 0; mt < Sh::NMT; ++mt) {
               float o[HW];

@@ -596,13 +596,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
         for (int si = 0; si < SB; ++si) m_new = fmaxf(m_new, lv[rb][si]);
         if (m_new == -INFINITY) continue;
-        const float sc = exp2f(mx[rb] - m_new);  // 0 when mx was -inf
+        // ex2.approx: these weights lie in [0, 1] and the merge is fp32 (relative error ~2^-22)
+        const float sc = fast_exp2(mx[rb] - m_new);  // 0 when mx was -inf
         sum[rb] *= sc;
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[rb][e] *= sc;
 #pragma unroll
         for (int si = 0; si < SB; ++si) {
-          const float wgt = exp2f(lv[rb][si] - m_new);  // 0 for absent segments
+          const float wgt = fast_exp2(lv[rb][si] - m_new);  // 0 for absent segments
           sum[rb] += wgt;
 #pragma unroll
           for (int e = 0; e < PER; ++e) acc[rb][e] += wgt * v[rb][si][e];
@@ -615,11 +616,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     for (int rb = 0; rb < RB; ++rb) {
       const int bl = r0 + rb, b = n0 + bl;
       if (bl >= NT) continue;
-      const float inv = sum[rb] > 0.f ? 1.f / sum[rb] : 0.f;
+      // sum >= 1 (the largest segment's own weight is 1): div.approx is within 2 ulp
+      const float inv = sum[rb] > 0.f ? __fdividef(1.f, sum[rb]) : 0.f;
 #pragma unroll
       for (int e = 0; e < PER; ++e) acc[rb][e] *= inv;
       if (b < p.batch && f0 == 0 && p.lse_out)  // one lane per (virtual) head
-        p.lse_out[(size_t)b * p.h + vhead] = nsg[rb] > 0 ? (mx[rb] + log2f(sum[rb])) * kLn2 : -INFINITY;
+        p.lse_out[(size_t)b * p.h + vhead] = nsg[rb] > 0 ? (mx[rb] + __log2f(sum[rb])) * kLn2 : -INFINITY;
       if constexpr (LATENT_ONLY) {
         if (b < p.batch) {
           float* dst = p.latent_out + ((size_t)b * p.h + head) * DB + lane * PER;
