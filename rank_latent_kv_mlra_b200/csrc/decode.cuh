@@ -852,40 +852,83 @@ __global__ void __launch_bounds__(Sh::THREADS, 1)
             warp_reduce_scatter<HW, false>(lt, lane);
             store_scattered<HW>(lt, red + q4 * HW, lane);
             named_bar_sync(bar_sync, 128);
-            // This runs while the next segment's tiles wait behind it, so it is kept short: an
-            // approximate reciprocal (l >= 1: the running maximum's own term contributes 1, so
-            // the 2-ulp bound of div.approx holds) and one lse store per warp, lane x holding
-            // head x, instead of one single-lane store per head.
-            static_assert(HW <= 32, "one lse lane per head");
-            float inv[HW];
-            float lse_lane = 0.f;
-#pragma unroll
-            for (int x = 0; x < HW; ++x) {
-              const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
-              inv[x] = __fdividef(Sh::FP8 ? p.o_scale : 1.f, l);
-              if (x == lane) lse_lane = m(x) + __log2f(l);
-            }
-            if (sw == 0 && lane < HW && hcol + lane < nheads)
-              p.lse_part[(size_t)slot * p.h + head0 + hcol + lane] = lse_lane;
-#pragma unroll
-            for (int mt = 0; mt < Sh::NMT; ++mt) {
-              float o[HW];
-              tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + hcol, o);
-              if constexpr (Sh::FP8) {
-                float o_lo[HW];
-                tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + NP + hcol, o_lo);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < HW; ++x) o[x] += o_lo[x];
-              } else {
-                tmem_ld_wait();
-              }
-              const int f = mt * 128 + row;
-              if (f < Sh::DB) {
-                float* dst = p.o_part + ((size_t)slot * p.h + head0 + hcol) * Sh::DB + f;
+            // This runs while the next segment's tiles wait behind it, so it is kept short: 1 / l
+            // by an approximate reciprocal (l >= 1: the running maximum's own term contributes 1,
+            // so the 2-ulp bound of div.approx holds), and each warp stores its lse values with
+            // one instruction, lane x holding head x.
+            if constexpr (HW >= 32 && Sh::NMT == 1) {
+              // 32 heads per warpgroup and one O tile: lane x of every warp works out head x's
+              // 1 / l and lse, and the O rows take 1 / l by shuffle (measured faster than every
+              // thread computing all 32; with several O tiles it is not)
+              static_assert(HW <= 32, "one lane per head");
+              float inv_lane = 0.f, lse_lane = 0.f;
+              {
+                float mv = 0.f;
 #pragma unroll
                 for (int x = 0; x < HW; ++x)
-                  if (hcol + x < nheads) dst[(size_t)x * Sh::DB] = o[x] * inv[x];
+                  if (x == lane) mv = m(x);
+                if (lane < HW) {
+                  const float l = red[lane] + red[HW + lane] + red[2 * HW + lane] + red[3 * HW + lane];
+                  inv_lane = __fdividef(Sh::FP8 ? p.o_scale : 1.f, l);
+                  lse_lane = mv + __log2f(l);
+                }
+              }
+              if (sw == 0 && lane < HW && hcol + lane < nheads)
+                p.lse_part[(size_t)slot * p.h + head0 + hcol + lane] = lse_lane;
+#pragma unroll
+              for (int mt = 0; mt < Sh::NMT; ++mt) {
+                float o[HW];
+                tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + hcol, o);
+                if constexpr (Sh::FP8) {
+                  float o_lo[HW];
+                  tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + NP + hcol, o_lo);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int x = 0; x < HW; ++x) o[x] += o_lo[x];
+                } else {
+                  tmem_ld_wait();
+                }
+                const int f = mt * 128 + row;
+                float* dst = p.o_part + ((size_t)slot * p.h + head0 + hcol) * Sh::DB + f;
+#pragma unroll
+                for (int x = 0; x < HW; ++x) {
+                  const float ix = __shfl_sync(0xffffffffu, inv_lane, x);
+                  if (f < Sh::DB && hcol + x < nheads) dst[(size_t)x * Sh::DB] = o[x] * ix;
+                }
+              }
+            } else {
+              // otherwise every thread works out 1 / l of each head itself
+              static_assert(HW <= 32, "one lse lane per head");
+              float inv[HW];
+              float lse_lane = 0.f;
+#pragma unroll
+              for (int x = 0; x < HW; ++x) {
+                const float l = red[x] + red[HW + x] + red[2 * HW + x] + red[3 * HW + x];
+                inv[x] = __fdividef(Sh::FP8 ? p.o_scale : 1.f, l);
+                if (x == lane) lse_lane = m(x) + __log2f(l);
+              }
+              if (sw == 0 && lane < HW && hcol + lane < nheads)
+                p.lse_part[(size_t)slot * p.h + head0 + hcol + lane] = lse_lane;
+#pragma unroll
+              for (int mt = 0; mt < Sh::NMT; ++mt) {
+                float o[HW];
+                tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + hcol, o);
+                if constexpr (Sh::FP8) {
+                  float o_lo[HW];
+                  tmem_load_row<HW>(tbase + lane_base + Sh::O_COL + mt * Sh::MN + NP + hcol, o_lo);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int x = 0; x < HW; ++x) o[x] += o_lo[x];
+                } else {
+                  tmem_ld_wait();
+                }
+                const int f = mt * 128 + row;
+                if (f < Sh::DB) {
+                  float* dst = p.o_part + ((size_t)slot * p.h + head0 + hcol) * Sh::DB + f;
+#pragma unroll
+                  for (int x = 0; x < HW; ++x)
+                    if (hcol + x < nheads) dst[(size_t)x * Sh::DB] = o[x] * inv[x];
+                }
               }
             }
             tc_fence_before();
