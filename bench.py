@@ -506,6 +506,22 @@ def run_ours(args, world, rank, local):
     # the pipelined steps computed the same output as the plain call
     assert torch.equal(out_host[(e2e_steps - 1) % NB], out.cpu())
 
+    # the same step through mlra_decode_noalloc (the library's fixed device scratch instead of
+    # a caller's workspace), timed the same way as the main leg
+    na_out = torch.empty_like(out)
+    na_args = (hdl, inp["q"], inp["pool"], inp["page_table"], inp["seq_lens"], na_out)
+    for _ in range(3):
+        M.mlra_decode_noalloc(*na_args)
+    n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    na_steps = max(20, args.steps // 4)
+    n0.record(stream)
+    for _ in range(na_steps):
+        M.mlra_decode_noalloc(*na_args)
+    n1.record(stream)
+    torch.cuda.synchronize()
+    noalloc_ms = n0.elapsed_time(n1) / na_steps
+    assert torch.equal(na_out, out)
+
     # the other configurations, each timed the same way in this run
     extra = {}
     if not args.headline_only:
@@ -532,6 +548,7 @@ def run_ours(args, world, rank, local):
 
     step_ms_max = max_over_ranks(step_ms, world, dev)
     e2e_ms_max = max_over_ranks(e2e_ms, world, dev)
+    noalloc_ms_max = max_over_ranks(noalloc_ms, world, dev)
     k_ms = [max_over_ranks(x, world, dev) for x in k_ms]
     if rank != 0:
         return
@@ -554,6 +571,8 @@ def run_ours(args, world, rank, local):
                 "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
                 "pipelined": "uploads, kernels and downloads of consecutive steps overlap on three streams",
                 "h2d_gbs_alone": h2d_gbs, "d2h_gbs_alone": d2h_gbs},
+        "noalloc": {"us_per_step": noalloc_ms_max * 1e3, "steps": na_steps,
+                    "note": "mlra_decode_noalloc on the same inputs (fixed library scratch, no workspace)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
