@@ -37,6 +37,13 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["value"] > 0
+    # the reference line describes its workload with the same keys as the GPU arm's line
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    w = W.WORKLOADS["mlra4_h8_b1_n256_f32"]
+    ours = bench.config_of(w, 2, line["config"]["cache_bytes_per_step"])
+    assert line["config"] == ours
 
 
 def _rank_main(rank, port, out):
