@@ -9,6 +9,8 @@ figures the pages state.
   (summed, k times the work; Table 2's MLRA-4 column, 4 n h d_c / 4 + 2 n h d_r per device,
   times the 4 devices).
 """
+import os
+
 import bench
 import workloads as W
 
@@ -45,3 +47,33 @@ def test_producer_bytes_match_the_oracle_count():
     w = W.WORKLOADS["mlra4_h128_b32_n8192"]
     for batch, d_model in [(32, 5120), (3, 256), (300, 384)]:
         assert bench.producer_bytes(w, batch, d_model) == P.bytes_per_step(batch, d_model, w.d_c, w.d_r)
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """A recorded ncu traffic figure stays attached to the decode kernel code it was measured
+    on: comment and blank-line edits and another shape's line keep the hash, a code edit
+    changes it."""
+    import shutil
+    src = os.path.join(bench.ROOT, "rank_latent_kv_mlra_b200", "csrc")
+    dst = tmp_path / "rank_latent_kv_mlra_b200" / "csrc"
+    dst.mkdir(parents=True)
+    for f in ("common.cuh", "decode.cuh", "mlra_api.cu"):
+        shutil.copy(os.path.join(src, f), dst / f)
+    w = W.WORKLOADS[W.HEADLINE]
+    base = bench.kernel_source_hash(w)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_source_hash(w) == base
+    with open(dst / "decode.cuh", "a") as fh:
+        fh.write("\n// a comment\n\n")
+    assert bench.kernel_source_hash(w) == base
+    api = (dst / "mlra_api.cu").read_text()
+    other = [l for l in api.splitlines() if l.startswith("using DecMla ")][0]
+    (dst / "mlra_api.cu").write_text(api.replace(other, other.replace("DecodeShape<", "DecodeShape< ")))
+    assert bench.kernel_source_hash(w) == base  # another shape's line
+    with open(dst / "decode.cuh", "a") as fh:
+        fh.write("static_assert(true, \"\");\n")
+    assert bench.kernel_source_hash(w) != base
+
+
+def test_recorded_traffic_is_reported_only_for_captured_workloads():
+    assert bench.recorded_traffic("mlra2sum_h128_b64_n4096") is None
