@@ -73,3 +73,29 @@ def test_host_argument_checks_return_codes(lib):
     assert lib.mlra_get_info(None, None) == -1
     assert lib.mlra_get_status(None, None) == -1
     lib.mlra_destroy(None)  # NULL-safe
+
+
+def test_host_checks_of_the_reading_and_cache_options(lib):
+    """The summed-blocks reading and the E4M3 cache are refused, before any CUDA call, for
+    shapes and settings that were not built or make no sense."""
+    P = ctypes.c_void_p
+    out = P()
+
+    def create(**kw):
+        f = dict(h=128, d_h=128, d_c=512, d_rope=64, k=4, page_size=64, softmax_scale=0.0,
+                 blocks_summed=0, attn_scale=0.0, cache_fp8=0, latent_scale=1.0, rope_scale=1.0)
+        f.update(kw)
+        cfg = M.mlra_config(*[f[n] for n, _ in M.mlra_config._fields_])
+        return lib.mlra_create(ctypes.byref(cfg), P(16), P(16), ctypes.byref(out))
+
+    assert create(blocks_summed=2) == -1                      # a flag: 0 or 1
+    assert create(cache_fp8=2) == -1
+    assert create(blocks_summed=1, k=1) == -2                 # summed reading: k = 2 or 4 only
+    assert create(cache_fp8=1, blocks_summed=1) == -2         # E4M3 with the partitioned MLRA-4 only
+    assert create(cache_fp8=1, k=2) == -2
+    assert create(cache_fp8=1, latent_scale=-1.0) == -1       # scales: finite and not negative
+    assert create(cache_fp8=1, rope_scale=float("inf")) == -1
+    assert create(cache_fp8=1, latent_scale=float("nan")) == -1
+    assert lib.mlra_create(None, P(16), P(16), ctypes.byref(out)) == -1
+    cfg = M.mlra_config(128, 128, 512, 64, 4, 64, 0.0)
+    assert lib.mlra_create(ctypes.byref(cfg), P(8), P(16), ctypes.byref(out)) == -1  # 16-byte aligned weights
